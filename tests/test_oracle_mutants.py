@@ -1,0 +1,47 @@
+"""Planted mistakes in copies of the oracle must each fail at least one pin.
+
+Each mutant is the oracle's C source with one plausible error written in
+(a dropped scale, an off-by-one mask, the wrong value columns, a wrong page or
+head index, a dropped max in lse, a sign slip in the merge).  The copy is
+compiled on the CPU into a temporary directory; the real oracle is untouched.
+"""
+import os
+
+import pytest
+
+import oracle
+from oracle_pins import ALL_PINS
+
+MUTANTS = {
+    "no_scale": ("s[j - first] = softmax_scale * acc;", "s[j - first] = acc;"),
+    "mask_off_by_one": ("int last = causal ? L - s_q + i : L - 1;",
+                        "int last = causal ? L - s_q + i - 1 : L - 1;"),
+    "value_from_rope_end": ("orow[c] += w * bf16_to_double(vrow[c]);",
+                            "orow[c] += w * bf16_to_double(vrow[c + (d - dv)]);"),
+    "page_index": ("block_table[(size_t)b * max_pages + j / page_size]",
+                   "block_table[(size_t)b * max_pages + 0 * (j / page_size)]"),
+    "slot_index": ("(size_t)(j % page_size)", "(size_t)((j + 1) % page_size)"),
+    "kv_head": ("const int g = h / heads_per_kv;", "const int g = h % h_kv;"),
+    "lse_drops_max": ("*lse_out = m + log(z);", "*lse_out = log(z);"),
+    "merge_sign": ("const double w = exp(part_lse[k] - total);",
+                   "const double w = exp(total - part_lse[k]);"),
+    "rope_dims_dropped": ("for (int c = 0; c < d; ++c) acc +=", "for (int c = 0; c < dv; ++c) acc +="),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(oracle.SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    path = os.path.join(tmp_path, f"mut_{name}.c")
+    with open(path, "w") as f:
+        f.write(src.replace(old, new))
+    lib = oracle.OracleLib(oracle.build(force=True, src=path, out=os.path.join(tmp_path, f"{name}.so")))
+    failures = []
+    for pin in ALL_PINS:
+        try:
+            pin(lib)
+        except (AssertionError, ValueError) as e:
+            failures.append(pin.__name__)
+    assert failures, f"mutant {name} passed every pin"
