@@ -1,0 +1,470 @@
+#!/usr/bin/env python
+"""Benchmark of the paged MLA decode hot path on B200.
+
+One *step* is one pass of the whole hot path over one batch: the length-balanced
+schedule (get_mla_metadata), the split-KV decode kernel and the merge kernel.
+The default workload is the uniform decode configuration (batch 64, s_q 1,
+128 query heads, 1 KV head, 576/512 dims, 4096 cached tokens each, 64-token
+pages in a shuffled 4096-page pool, bf16 N(0,1) data, scale 1/sqrt(192)).  Its
+inputs (302 MB of KV cache) are larger than the 126 MB L2, so no flush is
+needed between steps; the merge partials and q are small and may stay in L2.
+
+Prints ONE JSON line on rank 0.  ``value`` is the whole-job KV-read bandwidth
+(GB/s): KV bytes of all ranks' steps / max-over-ranks device time of the K
+timed steps.  Each step is replayed from a CUDA graph holding the three kernel
+launches.  ``roofline`` reports the decode call (split-KV kernel + merge
+kernel), timed per launch with CUDA events inside the timed region, against
+the measured HBM or bf16 peak.  ``e2e`` times the same step through the public
+Python API from pinned host buffers (inputs copied in, o and lse copied out
+every step).  ``cpu_baseline`` times the fp64 oracle on the host cores on a
+bounded sample of the same workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+    python bench.py --impl reference ...     # the oracle as the reference arm
+    python bench.py --all-configs            # one line per configuration (stderr + file)
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import mla_workloads as W  # noqa: E402
+
+METRIC = "MLA decode TFLOPS & KV-read GB/s vs B200 roofline; µs per decode call"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def work_counts(inp: dict) -> dict:
+    """Algorithmic bytes and flops of one decode call.
+
+    Bytes: every cached row a query row can see, read once (576 bf16 per token
+    per KV head), plus q read, o written (bf16) and lse written (fp32).  Split
+    partials, page-tail padding and L2 re-reads are not algorithmic.
+    Flops: 2 * (576 + 512) per (query row, visible token) pair.
+    """
+    lens = inp["cache_seqlens"].astype(np.int64)
+    s_q, h_q, h_kv, b = inp["s_q"], inp["h_q"], inp["h_kv"], inp["batch"]
+    kv_bytes = int(lens.sum()) * h_kv * W.D_QK * 2
+    if inp["causal"]:
+        vis = sum(int(np.clip(lens - (s_q - 1 - i), 0, None).sum()) for i in range(s_q))
+    else:
+        vis = int(lens.sum()) * s_q
+    flops = 2 * (W.D_QK + W.D_V) * h_q * vis
+    io_bytes = b * s_q * h_q * (W.D_QK * 2 + W.D_V * 2 + 4)
+    return dict(kv_bytes=kv_bytes, bytes=kv_bytes + io_bytes, flops=flops, tokens=int(lens.sum()))
+
+
+def roofline_time(wc, peaks, sustained=False):
+    t_hbm = wc["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    tf = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    t_tc = wc["flops"] / (tf * 1e12)
+    return (t_hbm, "hbm") if t_hbm >= t_tc else (t_tc, "tensor")
+
+
+def workload_desc(w: W.Workload) -> str:
+    return (f"{w.name} decode: batch={w.batch} s_q={w.s_q} h_q={w.h_q} h_kv={w.h_kv} d=576 dv=512 "
+            f"page=64 causal={w.causal} lengths={w.seqlen_kind}{list(w.seqlen_args)} bf16 N(0,1)")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.ok = [], 0, False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report nothing rather than guess
+            log("clock sampling unavailable:", e)
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return None
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        med = float(np.median(self.samples)) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- our arm
+def bench_ours(args, rank, world, local_rank):
+    import torch
+    import paged_mla_attention_b200 as pm
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = W.WORKLOADS[args.config]
+    inp = W.make_inputs(w, seed=w.seed + 1000 * rank)   # weak scaling: each rank its own batch
+    wc = work_counts(inp)
+    peaks, peaks_src = load_peaks()
+
+    def up(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+    host = dict(q=up(inp["q"]).pin_memory(), kvcache=up(inp["kvcache"]).pin_memory(),
+                block_table=torch.from_numpy(inp["block_table"]).pin_memory(),
+                cache_seqlens=torch.from_numpy(inp["cache_seqlens"]).pin_memory())
+    d = {k: v.to(dev) for k, v in host.items()}
+    R = inp["s_q"] * inp["h_q"] // inp["h_kv"]
+    o = torch.empty((inp["batch"], inp["s_q"], inp["h_q"], W.D_V), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((inp["batch"], inp["h_q"], inp["s_q"]), dtype=torch.float32, device=dev)
+    ws = torch.empty((pm.workspace_bytes(inp["batch"], inp["s_q"], inp["h_q"], inp["h_kv"]),),
+                     dtype=torch.uint8, device=dev)
+
+    meta_holder = {}
+
+    def step_meta():
+        meta_holder["m"], meta_holder["s"] = pm.get_mla_metadata(d["cache_seqlens"], R, inp["h_kv"])
+
+    def step_decode():
+        pm.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], W.D_V,
+                                  meta_holder["m"], meta_holder["s"],
+                                  softmax_scale=inp["softmax_scale"], causal=inp["causal"],
+                                  out=(o, lse), workspace=ws)
+
+    if args.profile:
+        # minimal plain-launch run for ncu: W warm-up steps then K steps, no graphs
+        for _ in range(args.warmup + args.steps):
+            step_meta()
+            step_decode()
+        torch.cuda.synchronize(dev)
+        err = pm.device_error()
+        if err:
+            raise RuntimeError(f"device error {err}")
+        return None, inp, wc
+
+    # warm-up (also compiles nothing: the library is prebuilt)
+    stream = torch.cuda.Stream(dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            step_meta()
+            step_decode()
+    torch.cuda.current_stream(dev).wait_stream(stream)
+    torch.cuda.synchronize(dev)
+    err = pm.device_error()
+    if err:
+        raise RuntimeError(f"device error {err} during warm-up")
+
+    # capture the step as two CUDA graphs (schedule | decode + merge)
+    g_meta, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_meta, stream=stream):
+        step_meta()
+    with torch.cuda.graph(g_dec, stream=stream):
+        step_decode()
+    for _ in range(3):
+        g_meta.replay()
+        g_dec.replay()
+    torch.cuda.synchronize(dev)
+
+    K = args.steps
+    ev_start = torch.cuda.Event(enable_timing=True)
+    ev_end = torch.cuda.Event(enable_timing=True)
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clk:
+        ev_start.record()
+        for k in range(K):
+            g_meta.replay()
+            ev_a[k].record()
+            g_dec.replay()
+            ev_b[k].record()
+        ev_end.record()
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = ev_start.elapsed_time(ev_end)
+    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]))
+    err = pm.device_error()
+    if err:
+        raise RuntimeError(f"device error {err} in the timed region")
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # end-to-end through the public API from pinned host buffers
+    e2e_steps = max(3, min(K, args.e2e_steps))
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+
+    def e2e_step():
+        dd = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+        m, s = pm.get_mla_metadata(dd["cache_seqlens"], R, inp["h_kv"])
+        oo, ll = pm.flash_mla_with_kvcache(dd["q"], dd["kvcache"], dd["block_table"],
+                                           dd["cache_seqlens"], W.D_V, m, s,
+                                           softmax_scale=inp["softmax_scale"], causal=inp["causal"])
+        o_h.copy_(oo, non_blocking=True)
+        lse_h.copy_(ll, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    # correctness spot-check of this very run against the oracle (rank 0, two sequences)
+    spot = None
+    if rank == 0 and not args.no_spot_check:
+        import oracle
+        from gpu_helpers import compare, subset
+        seqs = [0, inp["batch"] - 1]
+        sub = subset(inp, seqs, list(range(0, inp["h_q"], 8)))
+        ro, rl = oracle.decode_inputs(sub)
+        og = o.float().cpu().numpy()[seqs][:, :, ::8].astype(np.float64)
+        lg = lse.cpu().numpy()[seqs][:, ::8].astype(np.float64)
+        spot = compare(og, lg, ro, rl, what="bench spot check")
+
+    per_step_s = elapsed_ms / 1e3 / K
+    value = world * wc["kv_bytes"] / per_step_s / 1e9
+    dec_s = dec_ms / 1e3
+    t_roof, bound = roofline_time(wc, peaks)
+    if bound == "hbm":
+        achieved = wc["bytes"] / dec_s / 1e9
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved = wc["flops"] / dec_s / 1e12
+        peak, unit = peaks["bf16_tflops"], "TFLOP/s"
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(elapsed_ms / K, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "global_batch": inp["batch"] * world,
+                   "kv_tokens_per_gpu": wc["tokens"], "parallelism": f"replicas x{world} (batch-sharded, no exchange)",
+                   "l2": "inputs (302 MB KV) larger than the 126 MB L2; no flush",
+                   "step": "schedule + split-KV decode + merge, replayed from CUDA graphs"},
+        "us_per_call": round(dec_ms * 1e3, 3),
+        "tflops": round(wc["flops"] / dec_s / 1e12, 2),
+        "kv_read_gbs_per_call": round(wc["kv_bytes"] / dec_s / 1e9, 1),
+        "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+                     "frac": round(achieved / peak, 4), "traffic": args.traffic,
+                     "kernel": "decode call: split-KV decode kernel + merge kernel",
+                     "peak_source": f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback",
+                     "roofline_us": round(t_roof * 1e6, 2),
+                     "frac_of_roofline_time": round(t_roof / dec_s, 4)},
+        "e2e": {"value": round(world * wc["kv_bytes"] / (e2e_ms / 1e3 / e2e_steps) / 1e9, 3), "unit": "GB/s",
+                "steps": e2e_steps, "ms_per_step": round(e2e_ms / e2e_steps, 4),
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": 3 * K,
+        "clocks": clk.summary(),
+    }
+    if spot is not None:
+        result["parity_spot_check"] = {k: float(f"{v:.4g}") for k, v in spot.items()}
+    return result, inp, wc
+
+
+def cpu_baseline(inp, wc, budget_s):
+    """The oracle as it stands, on the host cores, on a bounded sample of the workload."""
+    import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from gpu_helpers import subset
+    order = list(range(inp["batch"]))
+    done_tokens, t_total, seqs_done = 0, 0.0, 0
+    for b in order:
+        sub = subset(inp, [b])
+        t = time.perf_counter()
+        oracle.decode_inputs(sub)
+        t_total += time.perf_counter() - t
+        done_tokens += int(inp["cache_seqlens"][b])
+        seqs_done += 1
+        if t_total >= budget_s:
+            break
+    frac = done_tokens / max(wc["tokens"], 1)
+    value = frac * wc["kv_bytes"] / t_total / 1e9
+    return {"value": round(value, 5), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{seqs_done} of {inp['batch']} sequences (all heads, all tokens), "
+                      f"{frac:.3f} of the workload's KV-token work, fp64, {t_total:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def bench_reference(args):
+    """The fp64 oracle on the host cores, timed on a bounded sample per step."""
+    import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from gpu_helpers import subset
+    w = W.WORKLOADS[args.config]
+    inp = W.make_inputs(w)
+    wc = work_counts(inp)
+    # size each step so that warm-up + timed steps take about `budget` seconds
+    probe = subset(inp, [0], [0, 1])
+    t = time.perf_counter()
+    oracle.decode_inputs(probe)
+    per_head = max((time.perf_counter() - t) / 2, 1e-5)
+    budget = args.reference_budget
+    heads = int(np.clip(budget / (args.steps + args.warmup) / per_head, 1, inp["h_q"]))
+    def one(k):
+        b = k % inp["batch"]
+        hs = [(k * heads + j) % inp["h_q"] for j in range(heads)]
+        sub = subset(inp, [b], sorted(set(hs)))
+        t0 = time.perf_counter()
+        oracle.decode_inputs(sub)
+        return time.perf_counter() - t0, int(inp["cache_seqlens"][b]) * len(set(hs))
+    for k in range(args.warmup):
+        one(k)
+    tt, work = 0.0, 0
+    for k in range(args.steps):
+        dt, wk = one(args.warmup + k)
+        tt += dt
+        work += wk
+    frac = work / (wc["tokens"] * inp["h_q"])
+    value = frac * wc["kv_bytes"] / tt / 1e9
+    sample = (f"each step: 1 sequence x {heads} of {inp['h_q']} heads (all tokens); "
+              f"{frac:.4f} of one workload's row-token work in total, fp64")
+    return {
+        "metric": METRIC, "value": round(value, 6), "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": workload_desc(w), "global_batch": inp["batch"]},
+        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="uniform", choices=list(W.WORKLOADS))
+    ap.add_argument("--all-configs", action="store_true",
+                    help="bench every configuration; one JSON line each on stderr and in --out")
+    ap.add_argument("--out", default=None)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--reference-budget", type=float, default=90.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-spot-check", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="plain launches only (warm-up + steps), for ncu; prints one short line")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="dram bytes per decode call from an ncu capture of the same kernels")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        print(json.dumps(bench_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        if args.profile:
+            bench_ours(args, rank, world, local_rank)
+            if rank == 0:
+                print(json.dumps({"profile_run": args.config, "steps": args.steps, "warmup": args.warmup}))
+            return
+        configs = list(W.WORKLOADS) if args.all_configs else [args.config]
+        main_name = "uniform" if args.all_configs else args.config
+        lines, main = [], None
+        for name in configs:
+            args.config = name
+            res, inp, wc = bench_ours(args, rank, world, local_rank)
+            lines.append(res)
+            if name == main_name:
+                main = (res, inp, wc)
+            if args.all_configs and rank == 0:
+                log(json.dumps(res))
+        res, inp, wc = main
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(inp, wc, args.cpu_budget)
+        if rank == 0:
+            if args.out:
+                with open(args.out, "w") as f:
+                    for r in lines:
+                        f.write(json.dumps(r) + "\n")
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,153 @@
+/*
+ * pagedmla.h - C ABI of the B200 (sm_100a) paged MLA decode library.
+ *
+ * The library decodes Multi-head Latent Attention over a paged KV cache, the
+ * operation that the DeepSeek FlashMLA pages describe:
+ *
+ *   - FlashMLA overview (deepseek.csdn.net), section 2.2 "DeepSeek-V3 MLA",
+ *     attention equation: o_{t,i} = sum_{j<=t} softmax_j(q_{t,i}.k_{j,i} /
+ *     sqrt(d_h + d_h^R)) v^C_{j,i}; only c^KV (512) and k^R (64) are cached,
+ *     the other projections are absorbed, so one cached 576-wide row is the
+ *     key of every query head and its first 512 entries are the value.
+ *   - same article, section 4.2(1): 64-token pages mapped through block_table;
+ *     a split-KV forward kernel plus a kernel that merges the splits.
+ *   - FlashMLA usage (blog.soe.dolphin-ai.jp), steps 3-4: the two calls
+ *     get_mla_metadata(cache_seqlens, s_q*h_q//h_kv, h_kv) and
+ *     flash_mla_with_kvcache(q, kvcache, block_table, cache_seqlens, dv,
+ *     tile_scheduler_metadata, num_splits, causal).
+ *
+ * Conventions for every entry point:
+ *   - Tensor arguments are DEVICE pointers to contiguous row-major buffers
+ *     owned by the caller; the library keeps no reference after returning.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  No entry point synchronises the host with the device and none
+ *     allocates device memory.
+ *   - The return value is PMLA_OK (0) or a negative PMLA_ERR_* code; nothing
+ *     is launched when an error is returned.  No C++ exception crosses the ABI.
+ *     pmla_last_error() gives a message for the last failing call of the
+ *     calling host thread.
+ *   - bf16 tensors are passed as pointers to 16-bit storage (uint16_t).
+ */
+#ifndef PAGEDMLA_H_
+#define PAGEDMLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PMLA_API __attribute__((visibility("default")))
+#else
+#define PMLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PMLA_OK 0
+#define PMLA_ERR_INVALID_ARG (-1)  /* null pointer, negative or inconsistent size      */
+#define PMLA_ERR_UNSUPPORTED (-2)  /* d != 576, dv != 512, no sm_100 device, ...      */
+#define PMLA_ERR_ALIGNMENT (-3)    /* a pointer is not 16-byte aligned                 */
+#define PMLA_ERR_CUDA (-4)         /* a CUDA runtime / driver call or launch failed    */
+#define PMLA_ERR_WORKSPACE (-5)    /* workspace pointer missing or too small           */
+#define PMLA_ERR_DEVICE (-6)       /* a kernel reported an error (see below)           */
+
+#define PMLA_PAGE_SIZE 64     /* tokens per KV page                                  */
+#define PMLA_HEAD_DIM 576     /* q / k width: 512 latent (c^KV) + 64 RoPE (k^R)      */
+#define PMLA_HEAD_DIM_V 512   /* value width: the latent part of the same row        */
+#define PMLA_METADATA_INTS 8  /* int32 entries per part in tile_scheduler_metadata   */
+
+/*
+ * Sizes for one batch shape, computed on the host from device properties.
+ *
+ *   batch, num_heads_per_head_k (= s_q * h_q / h_kv), num_heads_k (= h_kv):
+ *       the shape the metadata is for.
+ *   num_parts (out): number of scheduler parts; tile_scheduler_metadata has
+ *       num_parts * PMLA_METADATA_INTS int32 entries, num_splits has batch+1.
+ *   workspace_bytes (out): device workspace mla_decode_with_kvcache needs for
+ *       split partial results of this shape (an upper bound over all lengths).
+ * Uses the current CUDA device.  Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ */
+PMLA_API int mla_get_metadata_sizes(int batch, int num_heads_per_head_k, int num_heads_k, int* num_parts,
+                           size_t* workspace_bytes);
+
+/*
+ * Length-balanced split-KV schedule (step 3 of the FlashMLA usage).
+ *
+ * Splits the pages of all sequences (ceil(cache_seqlens[b] / 64) each) into
+ * num_parts contiguous ranges of roughly equal cost, charging each piece of a
+ * sequence a fixed overhead, so that one long sequence is shared by many SMs
+ * and many short ones are packed together.  Runs as one small kernel on
+ * `stream`; the host never reads the lengths.
+ *
+ *   cache_seqlens          int32 [batch], device, lengths in tokens (>= 0).
+ *   tile_scheduler_metadata int32 [num_parts][8], device, out.  Part p covers,
+ *       in (sequence, page) order, from (m[0], m[1]) up to but excluding
+ *       (m[2], m[3]); m[4] is the ordinal of its first piece among the pieces
+ *       of sequence m[0]; m[5..7] are 0.
+ *   num_splits             int32 [batch+1], device, out: exclusive prefix sum
+ *       of pieces per sequence (0 pieces: empty sequence, 1: unsplit).
+ *   num_parts              from mla_get_metadata_sizes for the same shape.
+ * Errors: INVALID_ARG, CUDA.
+ */
+PMLA_API int mla_get_metadata(const int32_t* cache_seqlens, int batch, int num_heads_per_head_k,
+                     int num_heads_k, int32_t* tile_scheduler_metadata, int num_parts,
+                     int32_t* num_splits, void* stream);
+
+/*
+ * Paged MLA decode (step 4 of the FlashMLA usage): for every sequence b,
+ * query token i < s_q and query head h, with g = h / (h_q / h_kv):
+ *
+ *   S_j   = softmax_scale * dot(q[b][i][h][0:576], K_j)   for visible j
+ *   lse   = log(sum_j exp(S_j))                           (natural log)
+ *   o     = sum_j exp(S_j - lse) * K_j[0:512]
+ *
+ * where K_j = kvcache[block_table[b][j / 64]][j % 64][g][0:576] and token j
+ * is visible when j < cache_seqlens[b] and, if causal, j <= cache_seqlens[b]
+ * - s_q + i.  A row that sees no token gets o = 0 and lse = -inf.
+ *
+ *   q             bf16 [batch][s_q][h_q][576]
+ *   kvcache       bf16 [num_pages][64][h_kv][576]
+ *   block_table   int32 [batch][max_pages_per_seq]; entries for pages a
+ *                 sequence uses must lie in [0, num_pages)
+ *   cache_seqlens int32 [batch], each <= 64 * max_pages_per_seq
+ *   tile_scheduler_metadata, num_parts, num_splits: from mla_get_metadata on
+ *                 the same cache_seqlens and shape (must not be modified
+ *                 before this call has run on the device)
+ *   o             bf16 [batch][s_q][h_q][512], out
+ *   lse           fp32 [batch][h_q][s_q], out
+ *   workspace     device scratch of >= workspace_bytes from
+ *                 mla_get_metadata_sizes; contents need not be initialised;
+ *                 must not be shared by calls that may run concurrently.
+ * Alignment: q, kvcache, o, workspace 16-byte aligned.
+ * Errors: INVALID_ARG, UNSUPPORTED (d != 576, dv != 512, h_q % h_kv != 0),
+ *         ALIGNMENT, WORKSPACE, CUDA.
+ * Device-side waits are bounded; a kernel that gives up records an error that
+ * pmla_device_error() returns.
+ */
+PMLA_API int mla_decode_with_kvcache(const uint16_t* q, const uint16_t* kvcache, const int32_t* block_table,
+                            const int32_t* cache_seqlens, int batch, int s_q, int h_q, int h_kv,
+                            int d, int dv, int num_pages, int max_pages_per_seq,
+                            const int32_t* tile_scheduler_metadata, int num_parts,
+                            const int32_t* num_splits, int causal, float softmax_scale,
+                            uint16_t* o, float* lse, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/*
+ * Reads and clears the device error word of the current device (synchronises
+ * the device).  Returns 0 if no kernel reported an error since the last call,
+ * else the kernel's error code (a positive number naming the wait that gave up).
+ */
+PMLA_API int pmla_device_error(void);
+
+/* Message for the last failing call of this host thread ("" if none). */
+PMLA_API const char* pmla_last_error(void);
+
+/* Library version string. */
+PMLA_API const char* pmla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDMLA_H_ */

@@ -1,0 +1,189 @@
+"""B200-native paged MLA decode: Python binding of libpagedmla.so.
+
+The two calls mirror the FlashMLA usage the DeepSeek pages show (usage steps
+3-4):
+
+    tile_scheduler_metadata, num_splits = get_mla_metadata(cache_seqlens, s_q * h_q // h_kv, h_kv)
+    o, lse = flash_mla_with_kvcache(q, kvcache, block_table, cache_seqlens, dv,
+                                    tile_scheduler_metadata, num_splits, causal=True)
+
+This module only marshals arguments: it checks tensor dtypes/devices, allocates
+the outputs and the split workspace with torch, and passes raw device pointers
+and the current CUDA stream to the C ABI (``include/pagedmla.h``).  Every step
+of the computation runs in the library's sm_100a kernels; there is no CPU or
+PyTorch fallback, and importing this module fails loudly if the library has not
+been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = ["get_mla_metadata", "flash_mla_with_kvcache", "device_error", "library", "LIB_PATH",
+           "PmlaError", "DEFAULT_SOFTMAX_SCALE"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedmla.so")
+PAGE_SIZE = 64
+HEAD_DIM = 576
+HEAD_DIM_V = 512
+METADATA_INTS = 8
+# 1 / sqrt(d_h + d_h^R) with d_h = 128, d_h^R = 64: the scale in the MLA
+# attention equation of the FlashMLA overview, section 2.2.
+DEFAULT_SOFTMAX_SCALE = 1.0 / math.sqrt(192.0)
+
+ERRORS = {-1: "invalid argument", -2: "unsupported", -3: "alignment", -4: "CUDA error",
+          -5: "workspace", -6: "device error"}
+
+
+class PmlaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"pagedmla error {code} ({ERRORS.get(code, '?')}): {msg}")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m paged_mla_attention_b200.build` (there is no fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.mla_get_metadata_sizes.argtypes = [I, I, I, ctypes.POINTER(I), ctypes.POINTER(SZ)]
+    lib.mla_get_metadata_sizes.restype = I
+    lib.mla_get_metadata.argtypes = [P, I, I, I, P, I, P, P]
+    lib.mla_get_metadata.restype = I
+    lib.mla_decode_with_kvcache.argtypes = [P, P, P, P] + [I] * 8 + [P, I, P, I, ctypes.c_float,
+                                                                     P, P, P, SZ, P]
+    lib.mla_decode_with_kvcache.restype = I
+    lib.pmla_device_error.argtypes = []
+    lib.pmla_device_error.restype = I
+    lib.pmla_last_error.argtypes = []
+    lib.pmla_last_error.restype = ctypes.c_char_p
+    lib.pmla_version.argtypes = []
+    lib.pmla_version.restype = ctypes.c_char_p
+    return lib
+
+
+library = _load()
+
+
+def _check(rc: int) -> None:
+    if rc != 0:
+        raise PmlaError(rc, library.pmla_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def metadata_sizes(batch: int, num_heads_per_head_k: int, num_heads_k: int) -> Tuple[int, int]:
+    """(num_parts, workspace_bytes) for this shape on the current device."""
+    parts = ctypes.c_int(0)
+    ws = ctypes.c_size_t(0)
+    _check(library.mla_get_metadata_sizes(batch, num_heads_per_head_k, num_heads_k,
+                                          ctypes.byref(parts), ctypes.byref(ws)))
+    return parts.value, ws.value
+
+
+def get_mla_metadata(cache_seqlens: torch.Tensor, num_heads_per_head_k: int,
+                     num_heads_k: int) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Length-balanced split-KV schedule for one decode step.
+
+    cache_seqlens: int32 [batch] on the GPU.  num_heads_per_head_k is
+    s_q * h_q // h_kv and num_heads_k is h_kv.  Returns
+    (tile_scheduler_metadata int32 [num_parts, 8], num_splits int32 [batch + 1]),
+    both on the GPU, computed on the current stream without a host sync.
+    """
+    _need(cache_seqlens, "cache_seqlens", torch.int32, 1)
+    batch = cache_seqlens.shape[0]
+    with torch.cuda.device(cache_seqlens.device):
+        parts, _ = metadata_sizes(batch, num_heads_per_head_k, num_heads_k)
+        meta = torch.empty((parts, METADATA_INTS), dtype=torch.int32, device=cache_seqlens.device)
+        splits = torch.empty((batch + 1,), dtype=torch.int32, device=cache_seqlens.device)
+        _check(library.mla_get_metadata(_ptr(cache_seqlens), batch, num_heads_per_head_k,
+                                        num_heads_k, _ptr(meta), parts, _ptr(splits),
+                                        _stream_ptr(cache_seqlens.device)))
+    return meta, splits
+
+
+def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: torch.Tensor,
+                           cache_seqlens: torch.Tensor, head_dim_v: int,
+                           tile_scheduler_metadata: torch.Tensor, num_splits: torch.Tensor,
+                           softmax_scale: Optional[float] = None, causal: bool = False,
+                           out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
+                           workspace: Optional[torch.Tensor] = None
+                           ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Paged MLA decode.
+
+    q           bf16 [batch, s_q, h_q, 576]
+    kvcache     bf16 [num_pages, 64, h_kv, 576]
+    block_table int32 [batch, max_pages]
+    cache_seqlens int32 [batch]
+    head_dim_v  512
+    Returns o bf16 [batch, s_q, h_q, 512] and lse fp32 [batch, h_q, s_q] (natural log).
+    softmax_scale defaults to 1/sqrt(192).  ``out`` and ``workspace`` may be
+    passed to avoid per-call allocation.
+    """
+    _need(q, "q", torch.bfloat16, 4)
+    _need(kvcache, "kvcache", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(cache_seqlens, "cache_seqlens", torch.int32, 1)
+    _need(tile_scheduler_metadata, "tile_scheduler_metadata", torch.int32, 2)
+    _need(num_splits, "num_splits", torch.int32, 1)
+    batch, s_q, h_q, d = q.shape
+    num_pages, page, h_kv, d2 = kvcache.shape
+    if page != PAGE_SIZE or d2 != d:
+        raise ValueError(f"kvcache must be [num_pages, {PAGE_SIZE}, h_kv, {d}], got {tuple(kvcache.shape)}")
+    if block_table.shape[0] != batch or cache_seqlens.shape[0] != batch or num_splits.shape[0] != batch + 1:
+        raise ValueError("batch size mismatch between q, block_table, cache_seqlens, num_splits")
+    if h_kv < 1 or h_q % h_kv:
+        raise ValueError("h_q must be a multiple of h_kv")
+    dev = q.device
+    for name, t in (("kvcache", kvcache), ("block_table", block_table), ("cache_seqlens", cache_seqlens),
+                    ("tile_scheduler_metadata", tile_scheduler_metadata), ("num_splits", num_splits)):
+        if t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, q on {dev}")
+    scale = DEFAULT_SOFTMAX_SCALE if softmax_scale is None else float(softmax_scale)
+    num_parts = tile_scheduler_metadata.shape[0]
+    with torch.cuda.device(dev):
+        _, ws_bytes = metadata_sizes(batch, s_q * (h_q // h_kv), h_kv)
+        if out is None:
+            o = torch.empty((batch, s_q, h_q, head_dim_v), dtype=torch.bfloat16, device=dev)
+            lse = torch.empty((batch, h_q, s_q), dtype=torch.float32, device=dev)
+        else:
+            o, lse = out
+        if workspace is None or workspace.numel() < ws_bytes:
+            workspace = torch.empty((max(ws_bytes, 16),), dtype=torch.uint8, device=dev)
+        _check(library.mla_decode_with_kvcache(
+            _ptr(q), _ptr(kvcache), _ptr(block_table), _ptr(cache_seqlens), batch, s_q, h_q, h_kv,
+            d, head_dim_v, num_pages, block_table.shape[1], _ptr(tile_scheduler_metadata), num_parts,
+            _ptr(num_splits), int(bool(causal)), scale, _ptr(o), _ptr(lse), _ptr(workspace),
+            workspace.numel(), _stream_ptr(dev)))
+    return o, lse
+
+
+def workspace_bytes(batch: int, s_q: int, h_q: int, h_kv: int) -> int:
+    return metadata_sizes(batch, s_q * (h_q // h_kv), h_kv)[1]
+
+
+def device_error() -> int:
+    """Read and clear the device error word (synchronises the current device)."""
+    return int(library.pmla_device_error())

@@ -1,0 +1,280 @@
+// extern "C" entry points of libpagedmla.so (declared in include/pagedmla.h).
+//
+// Argument checks happen here, on the host, before anything is launched; the
+// kernels themselves only defend against device-side data they cannot check
+// (page ids out of range, lost arrivals) and report through the device error
+// word instead of faulting.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include <cudaTypedefs.h>
+
+#include "../../include/pagedmla.h"
+#include "pagedmla_internal.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+__device__ int g_device_error;  // first error code any kernel reported
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int fail_cuda(cudaError_t e, const char* what) {
+  return fail(PMLA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceInfo {
+  bool ready = false;
+  int max_clusters = 0;
+  int* err_ptr = nullptr;
+};
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+
+// Per-device one-time set-up: kernel attributes, cluster occupancy, the
+// address of the device error word.  Returns 0 or a PMLA error.
+int device_setup(int* device_out, DeviceInfo** info_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(PMLA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    cudaDeviceProp prop;
+    e = cudaGetDeviceProperties(&prop, dev);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaGetDeviceProperties");
+    if (prop.major != 10 || prop.minor != 0)
+      return fail(PMLA_ERR_UNSUPPORTED, "needs an sm_100 (B200-class) GPU, device %d is sm_%d%d",
+                  dev, prop.major, prop.minor);
+    if ((size_t)prop.sharedMemPerBlockOptin < pmla::decode_smem_bytes())
+      return fail(PMLA_ERR_UNSUPPORTED, "device offers %zu B shared memory per block, need %zu",
+                  (size_t)prop.sharedMemPerBlockOptin, pmla::decode_smem_bytes());
+    int n = 0;
+    int rc = pmla::decode_max_active_clusters(dev, &n);
+    if (rc != 0) return fail_cuda((cudaError_t)rc, "cudaOccupancyMaxActiveClusters");
+    if (n < 1) return fail(PMLA_ERR_UNSUPPORTED, "decode kernel cannot be resident on this device");
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_device_error);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress(device error word)");
+    d.max_clusters = n;
+    d.err_ptr = static_cast<int*>(p);
+    d.ready = true;
+  }
+  *device_out = dev;
+  *info_out = &d;
+  return PMLA_OK;
+}
+
+int check_shape(int batch, int num_heads_per_head_k, int num_heads_k) {
+  if (batch < 0 || batch > 65535) return fail(PMLA_ERR_INVALID_ARG, "batch %d not in [0, 65535]", batch);
+  if (num_heads_per_head_k < 1 || num_heads_k < 1 || num_heads_k > 65535)
+    return fail(PMLA_ERR_INVALID_ARG, "bad head counts (%d per KV head, %d KV heads)",
+                num_heads_per_head_k, num_heads_k);
+  return PMLA_OK;
+}
+
+int parts_for(const DeviceInfo& d, int num_heads_per_head_k, int num_heads_k) {
+  const int n_rg = (num_heads_per_head_k + pmla::kRows - 1) / pmla::kRows;
+  const long long groups = (long long)n_rg * num_heads_k;
+  long long parts = d.max_clusters / groups;
+  return (int)(parts < 1 ? 1 : parts);
+}
+
+size_t workspace_for(int batch, int R, int h_kv, int num_parts, size_t* lse_offset) {
+  const size_t slots = (size_t)batch + (size_t)num_parts;
+  const size_t rows = slots * (size_t)h_kv * (size_t)R;
+  const size_t o_bytes = rows * pmla::kDV * sizeof(float);
+  *lse_offset = o_bytes;
+  return o_bytes + ((rows * sizeof(float) + 255) & ~size_t(255));
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pmla_version(void) { return "pagedmla 0.1.0 (sm_100a)"; }
+
+const char* pmla_last_error(void) { return g_last_error.c_str(); }
+
+int mla_get_metadata_sizes(int batch, int num_heads_per_head_k, int num_heads_k, int* num_parts,
+                           size_t* workspace_bytes) {
+  g_last_error.clear();
+  if (!num_parts || !workspace_bytes) return fail(PMLA_ERR_INVALID_ARG, "null output pointer");
+  int rc = check_shape(batch, num_heads_per_head_k, num_heads_k);
+  if (rc) return rc;
+  int dev;
+  DeviceInfo* d;
+  rc = device_setup(&dev, &d);
+  if (rc) return rc;
+  *num_parts = parts_for(*d, num_heads_per_head_k, num_heads_k);
+  size_t lse_off;
+  *workspace_bytes = workspace_for(batch, num_heads_per_head_k, num_heads_k, *num_parts, &lse_off);
+  return PMLA_OK;
+}
+
+int mla_get_metadata(const int32_t* cache_seqlens, int batch, int num_heads_per_head_k,
+                     int num_heads_k, int32_t* tile_scheduler_metadata, int num_parts,
+                     int32_t* num_splits, void* stream) {
+  g_last_error.clear();
+  int rc = check_shape(batch, num_heads_per_head_k, num_heads_k);
+  if (rc) return rc;
+  if (!tile_scheduler_metadata || !num_splits || (batch > 0 && !cache_seqlens))
+    return fail(PMLA_ERR_INVALID_ARG, "null pointer argument");
+  if (num_parts < 1) return fail(PMLA_ERR_INVALID_ARG, "num_parts %d < 1", num_parts);
+  cudaError_t e = pmla::launch_metadata(cache_seqlens, batch, num_parts, tile_scheduler_metadata,
+                                        num_splits, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "metadata kernel launch");
+  return PMLA_OK;
+}
+
+int mla_decode_with_kvcache(const uint16_t* q, const uint16_t* kvcache, const int32_t* block_table,
+                            const int32_t* cache_seqlens, int batch, int s_q, int h_q, int h_kv,
+                            int d, int dv, int num_pages, int max_pages_per_seq,
+                            const int32_t* tile_scheduler_metadata, int num_parts,
+                            const int32_t* num_splits, int causal, float softmax_scale,
+                            uint16_t* o, float* lse, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  g_last_error.clear();
+  if (d != PMLA_HEAD_DIM || dv != PMLA_HEAD_DIM_V)
+    return fail(PMLA_ERR_UNSUPPORTED, "head dims must be d=576, dv=512 (got %d, %d)", d, dv);
+  if (batch < 0 || batch > 65535 || s_q < 1 || h_q < 1 || h_kv < 1 || h_kv > 65535)
+    return fail(PMLA_ERR_INVALID_ARG, "bad shape batch=%d s_q=%d h_q=%d h_kv=%d", batch, s_q, h_q,
+                h_kv);
+  if (h_q % h_kv != 0)
+    return fail(PMLA_ERR_UNSUPPORTED, "h_q (%d) must be a multiple of h_kv (%d)", h_q, h_kv);
+  if (num_pages < 1 || max_pages_per_seq < 1 || num_parts < 1)
+    return fail(PMLA_ERR_INVALID_ARG, "num_pages, max_pages_per_seq and num_parts must be >= 1");
+  if ((long long)num_pages * pmla::kPage * h_kv > (1ll << 31))
+    return fail(PMLA_ERR_UNSUPPORTED, "kv cache too large for 32-bit row coordinates");
+  if (!std::isfinite(softmax_scale) || softmax_scale < 0.f)
+    return fail(PMLA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  if (!q || !kvcache || !block_table || !cache_seqlens || !tile_scheduler_metadata ||
+      !num_splits || !o || !lse)
+    return fail(PMLA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(q) || !aligned16(kvcache) || !aligned16(o))
+    return fail(PMLA_ERR_ALIGNMENT, "q, kvcache and o must be 16-byte aligned");
+  const long long R = (long long)s_q * (h_q / h_kv);
+  if (R > (1 << 20)) return fail(PMLA_ERR_UNSUPPORTED, "s_q * h_q / h_kv too large");
+  size_t lse_off;
+  const size_t need = workspace_for(batch, (int)R, h_kv, num_parts, &lse_off);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(PMLA_ERR_WORKSPACE, "workspace needs %zu bytes, 16-byte aligned (got %zu)", need,
+                workspace_bytes);
+  if (batch == 0) return PMLA_OK;
+
+  int dev;
+  DeviceInfo* info;
+  int rc = device_setup(&dev, &info);
+  if (rc) return rc;
+  auto encode = get_encode();
+  if (!encode) return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+
+  // kvcache as a 3-D tensor: [576 columns] x [h_kv heads] x [num_pages*64 tokens];
+  // each TMA box is 64 columns x 1 head x 64 tokens with the 128-byte swizzle.
+  CUtensorMap tmap;
+  cuuint64_t gdim[3] = {(cuuint64_t)pmla::kD, (cuuint64_t)h_kv,
+                        (cuuint64_t)num_pages * pmla::kPage};
+  cuuint64_t gstride[2] = {(cuuint64_t)pmla::kD * 2, (cuuint64_t)h_kv * pmla::kD * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)pmla::kPage};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult cr = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(kvcache),
+                       gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)cr);
+
+  pmla::DecodeParams p;
+  p.q = q;
+  p.block_table = block_table;
+  p.seqlens = cache_seqlens;
+  p.meta = tile_scheduler_metadata;
+  p.num_splits = num_splits;
+  p.o = o;
+  p.lse = lse;
+  p.part_o = static_cast<float*>(workspace);
+  p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + lse_off);
+  p.err = info->err_ptr;
+  p.batch = batch;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  p.h_kv = h_kv;
+  p.hpk = h_q / h_kv;
+  p.R = (int)R;
+  p.n_rg = (int)((R + pmla::kRows - 1) / pmla::kRows);
+  p.num_parts = num_parts;
+  p.max_pages = max_pages_per_seq;
+  p.num_pages = num_pages;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  if ((long long)num_parts * h_kv * p.n_rg > (1ll << 30))
+    return fail(PMLA_ERR_UNSUPPORTED, "grid too large");
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = pmla::decode_prepare(dev);
+  if (e != cudaSuccess) return fail_cuda(e, "decode kernel attributes");
+  e = pmla::launch_decode(p, tmap, st);
+  if (e != cudaSuccess) return fail_cuda(e, "decode kernel launch");
+
+  pmla::CombineParams c;
+  c.num_splits = num_splits;
+  c.part_o = p.part_o;
+  c.part_lse = p.part_lse;
+  c.o = o;
+  c.lse = lse;
+  c.batch = batch;
+  c.s_q = s_q;
+  c.h_q = h_q;
+  c.h_kv = h_kv;
+  c.hpk = p.hpk;
+  c.R = p.R;
+  e = pmla::launch_combine(c, st);
+  if (e != cudaSuccess) return fail_cuda(e, "combine kernel launch");
+  return PMLA_OK;
+}
+
+int pmla_device_error(void) {
+  int dev;
+  DeviceInfo* info;
+  int rc = device_setup(&dev, &info);
+  if (rc) return rc;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return fail_cuda(e, "cudaDeviceSynchronize");
+  int v = 0, zero = 0;
+  e = cudaMemcpy(&v, info->err_ptr, sizeof v, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail_cuda(e, "reading the device error word");
+  e = cudaMemcpy(info->err_ptr, &zero, sizeof zero, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return fail_cuda(e, "clearing the device error word");
+  return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// Internal definitions shared by the kernels and the C-ABI layer.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace pmla {
+
+constexpr int kPage = 64;       // tokens per page
+constexpr int kD = 576;         // q/k width
+constexpr int kDV = 512;        // value width
+constexpr int kRows = 128;      // query rows per tile (the MMA's M)
+constexpr int kMetaInts = 8;    // int32 per scheduler part
+
+// Fixed cost, in pages, that the scheduler charges every piece of a sequence:
+// loading the 128x576 query tile (144 KB, two pages' worth of bytes), the
+// epilogue drain of the 128x512 accumulator, and for split pieces the partial
+// write and its re-read by the merge kernel.
+constexpr int kPieceCostPages = 3;
+
+// Device error codes written by bounded waits that time out (first one wins).
+enum DeviceError : int {
+  kErrNone = 0,
+  kErrBadSmemAlign = 1,
+  kErrBadPage = 2,
+  kErrWaitBase = 100,  // + the id of the wait that gave up
+};
+
+struct DecodeParams {
+  const uint16_t* q;            // [b][s_q][h_q][576]
+  const int32_t* block_table;   // [b][max_pages]
+  const int32_t* seqlens;       // [b]
+  const int32_t* meta;          // [num_parts][8]
+  const int32_t* num_splits;    // [b+1]
+  uint16_t* o;                  // [b][s_q][h_q][512]
+  float* lse;                   // [b][h_q][s_q]
+  float* part_o;                // [slots][h_kv][R][512]
+  float* part_lse;              // [slots][h_kv][R]
+  int* err;                     // device error word
+  int batch, s_q, h_q, h_kv;
+  int hpk;                      // h_q / h_kv
+  int R;                        // s_q * hpk rows per KV head
+  int n_rg;                     // ceil(R / 128) row groups
+  int num_parts, max_pages, num_pages, causal;
+  float scale_log2;             // softmax_scale * log2(e)
+};
+
+struct CombineParams {
+  const int32_t* num_splits;
+  const float* part_o;
+  const float* part_lse;
+  uint16_t* o;
+  float* lse;
+  int batch, s_q, h_q, h_kv, hpk, R;
+};
+
+// Host launchers (each returns the CUDA error of its launch).
+cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* meta,
+                            int32_t* num_splits, cudaStream_t stream);
+cudaError_t decode_prepare(int device);  // one-time per-device kernel attributes
+int decode_max_active_clusters(int device, int* out);
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, cudaStream_t stream);
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
+size_t decode_smem_bytes();
+
+}  // namespace pmla

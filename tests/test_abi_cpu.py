@@ -1,0 +1,79 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects bad
+arguments with error codes before touching a GPU (CPU only: no compute)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedmla.h")
+LIB = os.path.join(ROOT, "paged_mla_attention_b200", "libpagedmla.so")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_mla_attention_b200 import build
+    build.build()
+    return ctypes.CDLL(LIB)
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"PMLA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_header_declares_entry_points():
+    names = declared_symbols()
+    for n in ["mla_get_metadata", "mla_get_metadata_sizes", "mla_decode_with_kvcache",
+              "pmla_device_error", "pmla_last_error", "pmla_version"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), f"{name} declared in pagedmla.h but not exported"
+
+
+def test_version(lib):
+    lib.pmla_version.restype = ctypes.c_char_p
+    assert b"sm_100a" in lib.pmla_version()
+
+
+def _decode(lib, **kw):
+    P, I = ctypes.c_void_p, ctypes.c_int
+    f = lib.mla_decode_with_kvcache
+    f.argtypes = [P, P, P, P] + [I] * 8 + [P, I, P, I, ctypes.c_float, P, P, P, ctypes.c_size_t, P]
+    f.restype = I
+    a = dict(q=0x10000, kv=0x20000, bt=0x30000, sl=0x40000, batch=2, s_q=1, h_q=16, h_kv=1,
+             d=576, dv=512, num_pages=8, max_pages=3, meta=0x50000, parts=4, splits=0x60000,
+             causal=0, scale=0.07, o=0x70000, lse=0x80000, ws=0x90000, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return f(a["q"], a["kv"], a["bt"], a["sl"], a["batch"], a["s_q"], a["h_q"], a["h_kv"], a["d"],
+             a["dv"], a["num_pages"], a["max_pages"], a["meta"], a["parts"], a["splits"], a["causal"],
+             a["scale"], a["o"], a["lse"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=575), -2), (dict(dv=256), -2), (dict(h_q=15, h_kv=2), -2),
+    (dict(batch=-1), -1), (dict(s_q=0), -1), (dict(num_pages=0), -1), (dict(parts=0), -1),
+    (dict(scale=float("nan")), -1), (dict(scale=-1.0), -1),
+    (dict(q=None), -1), (dict(lse=None), -1), (dict(splits=None), -1),
+    (dict(q=0x10001), -3), (dict(o=0x70008), -3), (dict(kv=0x20002), -3),
+    (dict(ws_bytes=16), -5), (dict(ws=None), -5), (dict(ws=0x90004), -5),
+])
+def test_decode_rejects_bad_arguments(lib, kw, code):
+    assert _decode(lib, **kw) == code
+    lib.pmla_last_error.restype = ctypes.c_char_p
+    assert lib.pmla_last_error()  # a message was recorded
+
+
+def test_metadata_rejects_bad_arguments(lib):
+    P, I = ctypes.c_void_p, ctypes.c_int
+    f = lib.mla_get_metadata
+    f.argtypes = [P, I, I, I, P, I, P, P]
+    f.restype = I
+    assert f(0x1000, -1, 128, 1, 0x2000, 4, 0x3000, None) == -1
+    assert f(0x1000, 4, 0, 1, 0x2000, 4, 0x3000, None) == -1
+    assert f(0x1000, 4, 128, 1, None, 4, 0x3000, None) == -1
+    assert f(0x1000, 4, 128, 1, 0x2000, 0, 0x3000, None) == -1

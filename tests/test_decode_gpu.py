@@ -1,0 +1,163 @@
+"""GPU parity: the sm_100a decode path (through the C ABI) against the fp64 oracle.
+
+Tolerances (spec parity bar, bf16 inputs / fp32 accumulation / bf16 o):
+max|o - o_ref| <= 1e-2, cosine(o, o_ref) >= 0.99999, max|lse - lse_ref| <= 1e-3.
+"""
+import numpy as np
+import pytest
+
+import mla_workloads as W
+import oracle
+from gpu_helpers import check_schedule, compare, run_gpu, subset, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _small(seqlens, s_q=1, h_q=128, h_kv=1, causal=False, seed=0, extra_pages=3, scale=W.SCALE_192):
+    w = W.Workload("case", len(seqlens), s_q, h_q, h_kv, causal, "explicit", (tuple(seqlens),),
+                   seed=seed, softmax_scale=scale)
+    return W.make_inputs(w, seqlens=seqlens, extra_pages=extra_pages)
+
+
+def _check(inp, what):
+    o, lse, meta, splits = run_gpu(inp)
+    ro, rl = oracle.decode_inputs(inp)
+    return compare(o, lse, ro, rl, what=what), meta, splits
+
+
+def test_tiny_config():
+    inp = W.make_inputs(W.WORKLOADS["tiny"])
+    stats, _, _ = _check(inp, "tiny")
+    assert stats["max_o"] < 4.0  # bf16 half-ulp of |o| stays under the o tolerance
+
+
+@pytest.mark.parametrize("h_q", [16, 64, 128])
+def test_page_boundary_lengths(h_q):
+    _check(_small([1, 63, 64, 65, 127, 128, 129, 200], h_q=h_q, seed=h_q), f"edges h_q={h_q}")
+
+
+def test_empty_and_single_token_sequences():
+    stats, _, splits = _check(_small([0, 1, 0, 70, 1], h_q=32, seed=5), "empty/single")
+    assert list(np.diff(splits)[[0, 2]]) == [0, 0]
+
+
+@pytest.mark.parametrize("s_q,h_q", [(2, 128), (2, 64), (3, 32), (4, 16)])
+def test_causal_multi_token(s_q, h_q):
+    # includes sequences shorter than s_q, whose first rows see nothing
+    _check(_small([1, 2, 3, 66, 130, 700], s_q=s_q, h_q=h_q, causal=True, seed=10 + s_q),
+           f"causal s_q={s_q} h_q={h_q}")
+
+
+def test_non_causal_multi_token():
+    _check(_small([5, 90, 300], s_q=2, h_q=64, causal=False, seed=21), "s_q=2 non-causal")
+
+
+def test_split_sequences_merge():
+    # long sequences next to short ones: pieces of the long ones go through the merge kernel
+    stats, meta, splits = _check(_small([9000, 100, 3000, 64, 1], h_q=128, seed=22), "splits")
+    assert np.diff(splits).max() >= 2, "expected at least one split sequence"
+
+
+def test_grouped_kv_heads():
+    _check(_small([70, 300, 5], s_q=1, h_q=32, h_kv=2, seed=23), "h_kv=2")
+    _check(_small([129, 40], s_q=2, h_q=64, h_kv=4, causal=True, seed=24), "h_kv=4 causal")
+
+
+def test_row_groups_beyond_128():
+    # s_q * h_q / h_kv = 256 and 192: two row groups per KV head
+    _check(_small([200, 1000], s_q=2, h_q=128, causal=True, seed=25), "R=256")
+    _check(_small([77, 513], s_q=3, h_q=64, causal=True, seed=26), "R=192")
+
+
+def test_zero_scale_gives_mean_of_values():
+    _check(_small([10, 150], h_q=16, seed=27, scale=0.0), "scale=0")
+
+
+def test_page_relabelling_is_bitwise_invariant():
+    inp = _small([300, 64, 1000], h_q=128, seed=28, extra_pages=9)
+    o1, l1, _, _ = run_gpu(inp)
+    perm = np.random.default_rng(7).permutation(inp["kvcache"].shape[0])
+    kv2 = np.empty_like(inp["kvcache"])
+    kv2[perm] = inp["kvcache"]
+    inp2 = dict(inp, kvcache=kv2, block_table=perm[inp["block_table"]].astype(np.int32))
+    o2, l2, _, _ = run_gpu(inp2)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_deterministic():
+    inp = _small([4000, 33, 1500], h_q=128, seed=29)
+    d = to_device(inp)
+    a = run_gpu(inp, dev_inputs=d)
+    b = run_gpu(inp, dev_inputs=d)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_lazy_rescale_path():
+    # q aligned with later keys so the running max climbs page after page:
+    # forces the O-row rescale command many times
+    inp = _small([64 * 12], h_q=128, seed=30)
+    kv = W.bf16_bits_to_f32(inp["kvcache"]).copy()
+    L = 64 * 12
+    t = np.arange(L)
+    pages = inp["block_table"][0][t // 64]
+    ramp = np.linspace(0.0, 6.0, L).astype(np.float32)  # scores grow along the sequence
+    kv[pages, t % 64, 0, :] *= 0.25
+    kv[pages, t % 64, 0, 570] = ramp * 40.0       # a RoPE column: not part of the values
+    q = W.bf16_bits_to_f32(inp["q"]).copy()
+    q[..., 570] = np.abs(q[..., 570]) + 1.0
+    inp["kvcache"] = W.f32_to_bf16_bits(kv)
+    inp["q"] = W.f32_to_bf16_bits(q)
+    _check(inp, "rescale")
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_scheduler_invariants(seed):
+    import torch
+    import paged_mla_attention_b200 as pm
+    rng = np.random.default_rng(1000 + seed)
+    for trial in range(20):
+        batch = int(rng.integers(1, 200))
+        kind = trial % 4
+        if kind == 0:
+            lens = rng.integers(0, 300, size=batch)
+        elif kind == 1:
+            lens = rng.integers(0, 40000, size=batch)
+        elif kind == 2:
+            lens = np.where(rng.random(batch) < 0.1, rng.integers(10000, 200000, size=batch),
+                            rng.integers(0, 100, size=batch))
+        else:
+            lens = np.full(batch, int(rng.integers(0, 5000)))
+        for heads in (16, 128, 256):
+            sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+            meta, splits = pm.get_mla_metadata(sl, heads, 1)
+            torch.cuda.synchronize()
+            check_schedule(meta.cpu().numpy(), splits.cpu().numpy(), lens, meta.shape[0])
+
+
+FULL = ["uniform", "varlen", "causal2", "skew"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_configs_sampled(name):
+    """Full-size workloads in the benchmark's launch configuration, checked on
+    sampled sequences (all their rows recomputed by the oracle) plus
+    properties that hold at any size."""
+    inp = W.make_inputs(W.WORKLOADS[name])
+    o, lse, meta, splits = run_gpu(inp)
+    lens = inp["cache_seqlens"]
+    check_schedule(meta, splits, lens, meta.shape[0])
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    vmax = float(np.abs(W.bf16_bits_to_f32(inp["kvcache"][..., :512])).max())
+    assert np.abs(o).max() <= vmax + 1e-2
+    # sampled sequences: the longest, the shortest, a split one, and a few random ones
+    rng = np.random.default_rng(5)
+    pick = {int(np.argmax(lens)), int(np.argmin(lens))}
+    multi = np.nonzero(np.diff(splits) >= 2)[0]
+    if multi.size:
+        pick.add(int(multi[len(multi) // 2]))
+    pick.update(int(x) for x in rng.choice(len(lens), size=min(3, len(lens)), replace=False))
+    heads = sorted(rng.choice(inp["h_q"], size=16, replace=False).tolist())
+    seqs = sorted(pick)
+    sub = subset(inp, seqs, heads)
+    ro, rl = oracle.decode_inputs(sub)
+    compare(o[seqs][:, :, heads], lse[seqs][:, heads], ro, rl, what=name)
