@@ -18,7 +18,7 @@
  *   Paged cache, same article section 4.2(1): logical 64-token blocks map to
  *   physical blocks through block_table.
  *
- * Readings where the pages leave a step open (each is listed in the design doc):
+ * Readings where the pages leave a step open:
  *   - query token i of s_q (0-based) sees cached tokens j <= L - s_q + i when
  *     causal, all j < L otherwise (the sum over j <= t, with the new tokens
  *     being the last s_q of the sequence);

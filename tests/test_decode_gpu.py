@@ -1,6 +1,6 @@
 """GPU parity: the sm_100a decode path (through the C ABI) against the fp64 oracle.
 
-Tolerances (spec parity bar, bf16 inputs / fp32 accumulation / bf16 o):
+Parity bar (bf16 inputs, fp32 accumulation, bf16 o):
 max|o - o_ref| <= 1e-2, cosine(o, o_ref) >= 0.99999, max|lse - lse_ref| <= 1e-3.
 """
 import numpy as np
