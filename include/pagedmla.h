@@ -134,6 +134,32 @@ PMLA_API int mla_decode_with_kvcache(const uint16_t* q, const uint16_t* kvcache,
                             void* stream);
 
 /*
+ * Allocation-free variant of mla_decode_with_kvcache (the FlashMLA pages have
+ * no counterpart: this entry point exists for callers that cannot allocate
+ * device memory, such as code inside a CUDA stream capture, runtimes that own
+ * all device memory up front, or plugins whose host forbids other allocations).
+ *
+ * Same arguments, meaning, layouts and errors as mla_decode_with_kvcache,
+ * without workspace/workspace_bytes: the split scratch comes from a 32 MiB
+ * array the library keeps in device memory (held on every GPU that loads the
+ * library, until the process exits).  Shapes whose scratch bound, as reported
+ * by mla_get_metadata_sizes, exceeds 32 MiB are rejected with
+ * PMLA_ERR_WORKSPACE and a message in pmla_last_error().
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * All calls share the array: calls whose work may overlap on the GPU race and
+ * must be serialised by the caller.  Allocates nothing.
+ */
+PMLA_API int mla_decode_with_kvcache_noalloc(const uint16_t* q, const uint16_t* kvcache,
+                                             const int32_t* block_table, const int32_t* cache_seqlens,
+                                             int batch, int s_q, int h_q, int h_kv, int d, int dv,
+                                             int num_pages, int max_pages_per_seq,
+                                             const int32_t* tile_scheduler_metadata, int num_parts,
+                                             const int32_t* num_splits, int causal,
+                                             float softmax_scale, uint16_t* o, float* lse,
+                                             void* stream);
+
+/*
  * Reads and clears the device error word of the current device (synchronises
  * the device).  Returns 0 if no kernel reported an error since the last call,
  * else the kernel's error code (a positive number naming the wait that gave up).

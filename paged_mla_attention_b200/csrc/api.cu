@@ -120,6 +120,10 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 
 }  // namespace
 
+namespace pmla {
+void set_last_error(const char* msg) { g_last_error = msg ? msg : ""; }
+}  // namespace pmla
+
 extern "C" {
 
 const char* pmla_version(void) { return "pagedmla 0.1.0 (sm_100a)"; }

@@ -65,4 +65,7 @@ cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, cud
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 size_t decode_smem_bytes();
 
+// Records the message pmla_last_error() returns on this host thread.
+void set_last_error(const char* msg);
+
 }  // namespace pmla
