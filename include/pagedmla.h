@@ -47,7 +47,7 @@ extern "C" {
 #define PMLA_OK 0
 #define PMLA_ERR_INVALID_ARG (-1)  /* null pointer, negative or inconsistent size      */
 #define PMLA_ERR_UNSUPPORTED (-2)  /* d != 576, dv != 512, no sm_100 device, ...      */
-#define PMLA_ERR_ALIGNMENT (-3)    /* a pointer is not 16-byte aligned                 */
+#define PMLA_ERR_ALIGNMENT (-3)    /* a pointer is not aligned as its argument requires */
 #define PMLA_ERR_CUDA (-4)         /* a CUDA runtime / driver call or launch failed    */
 #define PMLA_ERR_WORKSPACE (-5)    /* workspace pointer missing or too small           */
 #define PMLA_ERR_DEVICE (-6)       /* a kernel reported an error (see below)           */
@@ -119,8 +119,9 @@ PMLA_API int mla_get_metadata(const int32_t* cache_seqlens, int batch, int num_h
  *   workspace     device scratch of >= workspace_bytes from
  *                 mla_get_metadata_sizes; contents need not be initialised;
  *                 must not be shared by calls that may run concurrently.
- * Alignment: q, kvcache, o, workspace 16-byte aligned.
- * Errors: INVALID_ARG, UNSUPPORTED (d != 576, dv != 512, h_q % h_kv != 0),
+ * Alignment: q and kvcache 16-byte aligned; o and workspace 32-byte aligned.
+ * Errors: INVALID_ARG, UNSUPPORTED (d != 576, dv != 512, h_q % h_kv != 0, or
+ *         h_q/h_kv neither a divisor of 128 that is >= 8 nor a multiple of 128),
  *         ALIGNMENT, WORKSPACE, CUDA.
  * Device-side waits are bounded; a kernel that gives up records an error that
  * pmla_device_error() returns.

@@ -37,6 +37,7 @@ int fail_cuda(cudaError_t e, const char* what) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 struct DeviceInfo {
   bool ready = false;
@@ -176,6 +177,14 @@ int mla_decode_with_kvcache(const uint16_t* q, const uint16_t* kvcache, const in
                 h_kv);
   if (h_q % h_kv != 0)
     return fail(PMLA_ERR_UNSUPPORTED, "h_q (%d) must be a multiple of h_kv (%d)", h_q, h_kv);
+  {
+    // the query tile is loaded by TMA in boxes of min(h_q/h_kv, 128) rows
+    const int hpk = h_q / h_kv;
+    const bool ok = hpk < pmla::kRows ? (pmla::kRows % hpk == 0 && hpk >= 8) : (hpk % pmla::kRows == 0);
+    if (!ok)
+      return fail(PMLA_ERR_UNSUPPORTED,
+                  "h_q/h_kv = %d: must divide 128 (and be >= 8) or be a multiple of 128", hpk);
+  }
   if (num_pages < 1 || max_pages_per_seq < 1 || num_parts < 1)
     return fail(PMLA_ERR_INVALID_ARG, "num_pages, max_pages_per_seq and num_parts must be >= 1");
   if ((long long)num_pages * pmla::kPage * h_kv > (1ll << 31))
@@ -185,14 +194,14 @@ int mla_decode_with_kvcache(const uint16_t* q, const uint16_t* kvcache, const in
   if (!q || !kvcache || !block_table || !cache_seqlens || !tile_scheduler_metadata ||
       !num_splits || !o || !lse)
     return fail(PMLA_ERR_INVALID_ARG, "null pointer argument");
-  if (!aligned16(q) || !aligned16(kvcache) || !aligned16(o))
-    return fail(PMLA_ERR_ALIGNMENT, "q, kvcache and o must be 16-byte aligned");
+  if (!aligned16(q) || !aligned16(kvcache) || !aligned32(o))
+    return fail(PMLA_ERR_ALIGNMENT, "q and kvcache must be 16-byte aligned, o 32-byte aligned");
   const long long R = (long long)s_q * (h_q / h_kv);
   if (R > (1 << 20)) return fail(PMLA_ERR_UNSUPPORTED, "s_q * h_q / h_kv too large");
   size_t lse_off;
   const size_t need = workspace_for(batch, (int)R, h_kv, num_parts, &lse_off);
-  if (!workspace || workspace_bytes < need || !aligned16(workspace))
-    return fail(PMLA_ERR_WORKSPACE, "workspace needs %zu bytes, 16-byte aligned (got %zu)", need,
+  if (!workspace || workspace_bytes < need || !aligned32(workspace))
+    return fail(PMLA_ERR_WORKSPACE, "workspace needs %zu bytes, 32-byte aligned (got %zu)", need,
                 workspace_bytes);
   if (batch == 0) return PMLA_OK;
 
@@ -216,6 +225,22 @@ int mla_decode_with_kvcache(const uint16_t* q, const uint16_t* kvcache, const in
                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)cr);
+
+  // q as a 2-D tensor: [576 columns] x [batch*s_q*h_q rows]; boxes of 64 columns
+  // x min(h_q/h_kv, 128) rows with the 128-byte swizzle.
+  CUtensorMap tmap_q;
+  {
+    const int hpk = h_q / h_kv;
+    cuuint64_t qdim[2] = {(cuuint64_t)pmla::kD, (cuuint64_t)batch * s_q * h_q};
+    cuuint64_t qstride[1] = {(cuuint64_t)pmla::kD * 2};
+    cuuint32_t qbox[2] = {64, (cuuint32_t)(hpk < pmla::kRows ? hpk : pmla::kRows)};
+    cuuint32_t qestride[2] = {1, 1};
+    cr = encode(&tmap_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(q), qdim,
+                qstride, qbox, qestride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS)
+      return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled (q) failed (%d)", (int)cr);
+  }
 
   pmla::DecodeParams p;
   p.q = q;
@@ -246,7 +271,7 @@ int mla_decode_with_kvcache(const uint16_t* q, const uint16_t* kvcache, const in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = pmla::decode_prepare(dev);
   if (e != cudaSuccess) return fail_cuda(e, "decode kernel attributes");
-  e = pmla::launch_decode(p, tmap, st);
+  e = pmla::launch_decode(p, tmap, tmap_q, st);
   if (e != cudaSuccess) return fail_cuda(e, "decode kernel launch");
 
   pmla::CombineParams c;

@@ -10,24 +10,33 @@
 // combine kernel (the "merge of split results" kernel the article names).
 //
 // Design (B200-specific; the Hopper design on the pages is prior art only).
-// One 128-row tile needs Q (128x576 bf16 = 288 TMEM columns as an MMA A
-// operand), S = QK^T (128x64 fp32, 64 columns, double-buffered) and the output
-// accumulator O (128x512 fp32 = all 512 TMEM columns).  That does not fit one
-// SM's TMEM, so each work unit runs on a 2-CTA cluster with split roles:
+// A 128-row tile needs the query (128x576 bf16), S = Q K^T (fp32) and the
+// output accumulator O (128x512 fp32 = all 512 TMEM columns of an SM).  That
+// does not fit one SM, so every work unit is a 2-CTA cluster with split roles:
 //
-//   CTA 0 ("S-CTA"): Q lives in TMEM; a TMA warp streams whole 64-token pages
-//     (9 chunks of 64 columns, 128B-swizzled) into a 3-stage ring; one thread
-//     issues S = Q K^T as 36 tcgen05 MMAs (M=128, N=64, K=16, A from TMEM)
-//     into a double-buffered TMEM tile; four softmax warps (one row per
-//     thread) read S, keep the running max/sum in fp32 with a lazy rescale
-//     (the reference max only moves when the page max exceeds it by 2^8), and
-//     write P = exp2(S*c - m) as bf16 straight into CTA 1's shared memory
-//     (distributed shared memory, in the swizzled K-major MMA layout).
-//   CTA 1 ("O-CTA"): a TMA warp streams the value part of the same pages
-//     (8 chunks); one thread issues O += P V as 8 MMAs (M=128, N=256, K=16,
-//     V MN-major) into the 512-column TMEM accumulator; four correction warps
-//     rescale O rows when the S-CTA moved a row's reference max, and run the
-//     epilogue (O / l -> bf16 o, or fp32 partials) at the end of each piece.
+//   CTA 0 ("S-CTA"): the latent part of Q (512 columns) lives in TMEM as an MMA
+//     A operand (256 columns), its RoPE part (64 columns) in shared memory; S
+//     is double-buffered in the other 2 x 128 TMEM columns.  A TMA warp
+//     streams 16 KB chunk stages through a 13-stage ring: chunk c of two
+//     consecutive pages (rows 0-63 page A, rows 64-127 page B, 64 columns,
+//     128B swizzle), so one MMA covers 128 tokens (N = 128 runs the tensor
+//     core at full rate, N = 64 does not).  One thread issues per page pair
+//     32 TS MMAs (latent, A from TMEM) + 4 SS MMAs (RoPE).  Four softmax warps
+//     (one row per thread) read S, apply the mask, keep the running max/sum in
+//     fp32 with a lazy rescale (the reference max only moves when a pair's max
+//     exceeds it by 2^8), and push P (bf16, swizzled K-major MMA layout) plus
+//     per-row factors into CTA 1's shared memory with st.async, which
+//     completes bytes on CTA 1's barrier: no fence, no extra arrival.
+//     The query tile itself arrives through the same ring (TMA), and the
+//     softmax warps copy its latent chunks into TMEM.
+//   CTA 1 ("O-CTA"): a TMA warp streams the value part of the same pages in
+//     32 KB half-page stages (mostly L2 hits: CTA 0 just read the page); one
+//     thread issues O += P V as 8 MMAs per page (M=128, N=256, K=16, V
+//     MN-major) into the 512-column accumulator; a relay warp re-arms each
+//     consumed P slot's barrier with its byte count and returns the slot to
+//     CTA 0; four correction warps rescale O rows when CTA 0 moved a row's
+//     reference max, and run the epilogue (O / l -> bf16 o, or fp32 partials)
+//     at the end of each piece.
 //
 // Every wait is bounded (see ptx.cuh); a timeout records an error code and
 // makes all roles leave their loops, drain their in-flight copies and MMAs,
@@ -39,43 +48,52 @@ namespace pmla {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kStages = 3;
-constexpr int kPSlots = 2;
-constexpr uint32_t kChunkBytes = 64 * 64 * 2;             // 64 tokens x 64 columns bf16
-constexpr uint32_t kKStageBytes = 9 * kChunkBytes;         // whole page row (576)
-constexpr uint32_t kVStageBytes = 8 * kChunkBytes;         // value part (512)
-constexpr uint32_t kPBytes = kRows * kPage * 2;            // 128 x 64 bf16
+constexpr int kThreads = 384;  // 4 role warps + two 4-warp groups
+constexpr int kRing = 10;                          // S-CTA chunk stages
+constexpr int kStageBufs = 2;                      // S-CTA P staging buffers
+constexpr uint32_t kChunkBytes = 128 * 64 * 2;     // 128 rows x 64 columns bf16
+constexpr uint32_t kPageChunkBytes = 64 * 64 * 2;  // one page's 64 tokens x 64 columns
+constexpr int kVStages = 4;                        // O-CTA half-page stages
+constexpr uint32_t kVStageBytes = 4 * kPageChunkBytes;  // 64 tokens x 256 columns
+constexpr int kPSlots = 4;
+constexpr uint32_t kPBytes = kRows * kPage * 2;    // 128 x 64 bf16
 
-struct SideSlot {        // per-P-slot row data sent by the S-CTA
-  uint32_t flags;        // bit0: some row moved its reference max; bit1: last page of piece
-  uint32_t pad[3];
+struct SideSlot {        // per-P-slot row data sent with every P tile
+  uint32_t wflag[4];     // per softmax warp: some row of the warp moved its reference max
   float alpha[kRows];    // O row rescale factors (1 = unchanged)
-  float linv[kRows];     // 1 / row sum, valid on the last page of a piece
+  float linv[kRows];     // 1 / (sum of rounded weights) so far; used on a piece's last page
 };
+constexpr uint32_t kSideBytes = sizeof(SideSlot);
+constexpr uint32_t kPFullTx = kPBytes + kSideBytes;  // bytes every P message carries
 
 struct Mailbox {         // MMA thread -> correction warps (O-CTA)
-  int cmd;               // 1: rescale rows by side slot `slot`; 2: epilogue
-  int slot;
+  int cmd;               // kCmdRescale or kCmdEpilogue
+  int slot;              // P slot whose alpha to apply (rescale)
   int b;
   int part_slot;         // partial slot index, or -1 for a direct write
   float linv[kRows];
 };
-
 enum : int { kCmdRescale = 1, kCmdEpilogue = 2 };
 
-// mbarrier indices (same offsets in both CTAs; meaning depends on the role)
+// mbarriers: one index space for both CTAs, each CTA initialises its own
 enum : int {
-  kBarFull = 0,       // [3] page stage loaded (TMA tx)
-  kBarEmpty = 3,      // [3] page stage consumed (MMA commit)
-  kBarSFull = 6,      // S-CTA [2]: S tile ready (commit) | O-CTA [2]: P slot consumed (commit)
-  kBarSFree = 8,      // S-CTA [2]: S tile read by softmax warps (128 arrivals)
-  kBarQFull = 10,     // S-CTA: Q tile in TMEM (128) | O-CTA: mailbox command posted (1)
-  kBarCmdDone = 11,   // O-CTA: command done (128)
-  kBarPFree = 12,     // S-CTA [2]: P slot free again (remote arrival from the O-CTA)
-  kBarPFull = 14,     // O-CTA [2]: P slot written (remote arrival from the S-CTA)
-  kBarDrain = 16,     // both: all issued MMAs complete
-  kNumBars = 17
+  kBarRingFull = 0,                      // S [13] chunk stage loaded (TMA tx)
+  kBarRingEmpty = kBarRingFull + kRing,  // S [13] chunk stage consumed
+  kBarSFull = kBarRingEmpty + kRing,     // S [2] S tile ready (commit)
+  kBarSFree = kBarSFull + 2,             // S [2] S tile read by softmax warps (128)
+  kBarQFull = kBarSFree + 2,             // S Q latent in TMEM (128)
+  kBarQrFull = kBarQFull + 1,            // S Q RoPE chunk loaded (TMA tx)
+  kBarQrEmpty = kBarQrFull + 1,          // S Q RoPE chunk no longer read (commit)
+  kBarPFree = kBarQrEmpty + 1,           // S [4] P slot free again (remote arrival)
+  kBarStageFree = kBarPFree + kPSlots,   // S [2] staging buffer copied out (remote arrival)
+  kBarVFull = kBarStageFree + kStageBufs,  // O [4] V half-stage loaded (TMA tx)
+  kBarVEmpty = kBarVFull + kVStages,     // O [4] V half-stage consumed (commit)
+  kBarPFull = kBarVEmpty + kVStages,     // O [4] P slot written (armed + st.async tx)
+  kBarPCons = kBarPFull + kPSlots,       // O [4] P slot consumed (commit)
+  kBarCmdFull = kBarPCons + kPSlots,     // O mailbox command posted (1)
+  kBarCmdDone = kBarCmdFull + 1,         // O command done (128)
+  kBarDrain = kBarCmdDone + 1,           // both: all issued MMAs complete
+  kNumBars = kBarDrain + 1
 };
 
 struct Ctrl {
@@ -84,24 +102,40 @@ struct Ctrl {
   int abort_flag;
 };
 
-constexpr uint32_t OFF_P = kStages * kVStageBytes;                          // O-CTA P slots
-constexpr uint32_t OFF_SIDE = OFF_P + kPSlots * kPBytes;
-constexpr uint32_t OFF_MAIL = OFF_SIDE + kPSlots * sizeof(SideSlot);
-constexpr uint32_t OFF_CTRL = (OFF_MAIL + sizeof(Mailbox) + 15u) & ~15u;
+// shared-memory layouts (offsets from a 1024-byte aligned base)
+constexpr uint32_t OFF_QROPE = 0;                                 // S-CTA: Q RoPE chunk
+constexpr uint32_t OFF_RING = kChunkBytes;                        // S-CTA: chunk ring
+constexpr uint32_t OFF_STAGE = OFF_RING + kRing * kChunkBytes;    // S-CTA: P staging
+constexpr uint32_t OFF_V = 0;                                     // O-CTA: V ring
+constexpr uint32_t OFF_P = OFF_V + kVStages * kVStageBytes;       // O-CTA: P slots
+constexpr uint32_t OFF_SIDE = OFF_P + kPSlots * kPBytes;          // O-CTA: side slots
+constexpr uint32_t OFF_MAIL = OFF_SIDE + kPSlots * kSideBytes;    // O-CTA: mailbox
+constexpr uint32_t OFF_STAGE_SIDE = OFF_STAGE + kStageBufs * kPBytes;  // S-CTA: staged side data
+constexpr uint32_t OFF_XCH = OFF_STAGE_SIDE + kStageBufs * kSideBytes;  // S-CTA: row exchange
+constexpr uint32_t kXchBytes = (2 * 2 * kRows + 2 * kRows + 2 * kRows) * 4;  // max x2 pairs, l, lr
+constexpr uint32_t OFF_CTRL = OFF_XCH + kXchBytes;                             // both
 constexpr uint32_t SMEM_BYTES = OFF_CTRL + sizeof(Ctrl);
-static_assert(kStages * kKStageBytes <= OFF_CTRL, "S-CTA ring overlaps the control block");
+static_assert(OFF_MAIL + sizeof(Mailbox) <= OFF_CTRL, "O-CTA regions overlap the control block");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget exceeded");
-static_assert(OFF_P % 1024 == 0, "P slots must be 1024-byte aligned for the 128B swizzle");
+static_assert(OFF_P % 1024 == 0 && OFF_RING % 1024 == 0 && OFF_STAGE % 1024 == 0,
+              "swizzled tiles need 1024-byte alignment");
+static_assert(OFF_SIDE % 16 == 0 && kSideBytes % 16 == 0, "side slots need 16-byte alignment");
 
 // TMEM column map
-constexpr uint32_t kTmemQ = 0;      // S-CTA: Q, 288 columns (bf16 pairs)
-constexpr uint32_t kTmemS = 288;    // S-CTA: two 64-column S tiles
+constexpr uint32_t kTmemQ = 0;      // S-CTA: latent Q, 256 columns of bf16 pairs
+constexpr uint32_t kTmemS = 256;    // S-CTA: two 128-column S tiles
 constexpr uint32_t kTmemO = 0;      // O-CTA: 512 columns
+
+constexpr float kLn2 = 0.69314718055994531f;
+constexpr float kTau = 8.0f;        // lazy rescale threshold (log2 units)
 
 struct Ring {
   uint32_t idx = 0, phase = 0;
   __device__ __forceinline__ void next(uint32_t n) {
     if (++idx == n) { idx = 0; phase ^= 1u; }
+  }
+  __device__ __forceinline__ void advance(uint32_t n, uint32_t by) {
+    for (uint32_t i = 0; i < by; ++i) next(n);
   }
 };
 
@@ -141,8 +175,38 @@ __device__ __forceinline__ int piece_slot(const DecodeParams& P, int b, int ordi
   return (s1 - s0 >= 2) ? s0 + ordinal : -1;
 }
 
+__device__ __forceinline__ int load_page(const DecodeParams& P, int b, int p) {
+  int page = P.block_table[(size_t)b * P.max_pages + p];
+  if (page < 0 || page >= P.num_pages) {
+    atomicCAS(P.err, 0, kErrBadPage);
+    page = P.num_pages;  // outside the tensor map: TMA fills zeros
+  }
+  return page;
+}
+
+// TMA the 64-column chunk c of this tile's 128 query rows into `dst`
+// (boxes of min(hpk,128) rows; rows past R are left untouched).  Returns bytes.
+__device__ __forceinline__ uint32_t load_q_chunk(const DecodeParams& P, const CUtensorMap* tmap_q,
+                                                 uint32_t dst, uint32_t bar, int b, int g, int rg,
+                                                 int c, uint64_t pol, bool issue) {
+  const int qbox = P.hpk < kRows ? P.hpk : kRows;
+  uint32_t bytes = 0;
+  for (int j = 0; j < kRows / qbox; ++j) {
+    const int rr0 = rg * kRows + j * qbox;
+    if (rr0 >= P.R) break;
+    if (issue) {
+      const int qi = rr0 / P.hpk;
+      const int row = (b * P.s_q + qi) * P.h_q + g * P.hpk + rr0 % P.hpk;
+      tma_load_2d(dst + (uint32_t)(j * qbox * 128), tmap_q, bar, c * 64, row, pol);
+    }
+    bytes += (uint32_t)qbox * 128u;
+  }
+  return bytes;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const DecodeParams P) {
+decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_q,
+              const DecodeParams P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x;
@@ -165,27 +229,48 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const DecodeParams P)
   auto bar = [&](int i) { return smem_u32(&ctrl->bar[i]); };
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(kBarFull + s), 1);
-      mbar_init(bar(kBarEmpty + s), 1);
+    if (rank == 0) {
+      for (int s = 0; s < kRing; ++s) {
+        mbar_init(bar(kBarRingFull + s), 1);
+        mbar_init(bar(kBarRingEmpty + s), 1);
+      }
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(bar(kBarSFull + s), 1);
+        mbar_init(bar(kBarSFree + s), 256);
+      }
+      mbar_init(bar(kBarQFull), 256);
+      mbar_init(bar(kBarQrFull), 1);
+      mbar_init(bar(kBarQrEmpty), 1);
+      for (int s = 0; s < kPSlots; ++s) mbar_init(bar(kBarPFree + s), 1);
+      for (int s = 0; s < kStageBufs; ++s) mbar_init(bar(kBarStageFree + s), 1);
+    } else {
+      for (int s = 0; s < kVStages; ++s) {
+        mbar_init(bar(kBarVFull + s), 1);
+        mbar_init(bar(kBarVEmpty + s), 1);
+      }
+      for (int s = 0; s < kPSlots; ++s) {
+        mbar_init(bar(kBarPFull + s), 1);
+        mbar_init(bar(kBarPCons + s), 1);
+      }
+      mbar_init(bar(kBarCmdFull), 1);
+      mbar_init(bar(kBarCmdDone), 256);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(kBarSFull + s), 1);
-      mbar_init(bar(kBarSFree + s), 128);
-      mbar_init(bar(kBarPFree + s), 1);
-      mbar_init(bar(kBarPFull + s), 1);
-    }
-    mbar_init(bar(kBarQFull), rank == 0 ? 128 : 1);
-    mbar_init(bar(kBarCmdDone), 128);
     mbar_init(bar(kBarDrain), 1);
     ctrl->abort_flag = 0;
     fence_mbar_init();
+    if (rank == 1) {
+      // arm every P slot for its first message (the relay re-arms after each use)
+      for (int s = 0; s < kPSlots; ++s) mbar_arrive_expect_tx(bar(kBarPFull + s), kPFullTx);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&ctrl->tmem_base), 512);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmap_kv);
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmap_kv);
+    tma_prefetch_desc(&tmap_q);
+  }
   tc_fence_before();
   __syncthreads();
   cluster_arrive();
@@ -198,136 +283,239 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const DecodeParams P)
   if (rank == 0) {
     // =========================================================== S-CTA
     if (warp == 0 && lane == 0) {
-      // ---- TMA producer: whole pages (9 chunks)
+      // ---- TMA producer: query chunks, then chunk c of each page pair
       Ring st;
-      bool ok = true;
-      uint32_t issued_phase[kStages];
-      bool issued[kStages] = {false, false, false};
-      const uint64_t pol = policy_evict_normal();
+      uint32_t qr_phase = 0;
+      bool ok = true, qr_issued = false;
+      uint32_t qr_issued_phase = 0;
+      uint32_t issued_phase[kRing];
+      bool issued[kRing];
+      for (int s = 0; s < kRing; ++s) issued[s] = false;
+      const uint64_t pol_q = policy_evict_last();
+      const uint64_t pol_kv = policy_evict_normal();
       for_each_piece(P, it, [&](int b, int p0, int p1, int) {
-        for (int p = p0; p < p1 && ok; ++p) {
-          ok = mbar_wait(bar(kBarEmpty + st.idx), st.phase ^ 1u, abortf, P.err, kErrWaitBase + 1);
-          if (!ok) break;
-          int page = P.block_table[(size_t)b * P.max_pages + p];
-          if (page < 0 || page >= P.num_pages) {
-            atomicCAS(P.err, 0, kErrBadPage);
-            page = P.num_pages;  // out of the tensor map: TMA fills zeros
-          }
-          const uint32_t fb = bar(kBarFull + st.idx);
-          mbar_arrive_expect_tx(fb, kKStageBytes);
-          const uint32_t dst = sbase + st.idx * kKStageBytes;
-#pragma unroll
-          for (int c = 0; c < 9; ++c)
-            tma_load_3d(dst + c * kChunkBytes, &tmap_kv, fb, c * 64, g, page * kPage, pol);
+        // latent query chunks 0..7 through the ring
+        for (int c = 0; c < 8; ++c) {
+          ok = mbar_wait(bar(kBarRingEmpty + st.idx), st.phase ^ 1u, abortf, P.err, kErrWaitBase + 1);
+          if (!ok) return false;
+          const uint32_t fb = bar(kBarRingFull + st.idx);
+          const uint32_t dst = sbase + OFF_RING + st.idx * kChunkBytes;
+          mbar_arrive_expect_tx(fb, load_q_chunk(P, &tmap_q, dst, fb, b, g, rg, c, pol_q, false));
+          load_q_chunk(P, &tmap_q, dst, fb, b, g, rg, c, pol_q, true);
           issued[st.idx] = true;
           issued_phase[st.idx] = st.phase;
-          st.next(kStages);
+          st.next(kRing);
         }
-        return ok;
+        // RoPE chunk 8 into its own buffer (freed when the piece's MMAs are done)
+        ok = mbar_wait(bar(kBarQrEmpty), qr_phase ^ 1u, abortf, P.err, kErrWaitBase + 2);
+        if (!ok) return false;
+        {
+          const uint32_t fb = bar(kBarQrFull);
+          mbar_arrive_expect_tx(fb, load_q_chunk(P, &tmap_q, sbase + OFF_QROPE, fb, b, g, rg, 8, pol_q, false));
+          load_q_chunk(P, &tmap_q, sbase + OFF_QROPE, fb, b, g, rg, 8, pol_q, true);
+          qr_issued = true;
+          qr_issued_phase = qr_phase;
+          qr_phase ^= 1u;
+        }
+        // page pairs
+        for (int pa = p0; pa < p1; pa += 2) {
+          const int npg = (pa + 1 < p1) ? 2 : 1;
+          const int pageA = load_page(P, b, pa);
+          const int pageB = npg == 2 ? load_page(P, b, pa + 1) : 0;
+          for (int c = 0; c < 9; ++c) {
+            ok = mbar_wait(bar(kBarRingEmpty + st.idx), st.phase ^ 1u, abortf, P.err, kErrWaitBase + 3);
+            if (!ok) return false;
+            const uint32_t fb = bar(kBarRingFull + st.idx);
+            const uint32_t dst = sbase + OFF_RING + st.idx * kChunkBytes;
+            mbar_arrive_expect_tx(fb, (uint32_t)npg * kPageChunkBytes);
+            tma_load_3d(dst, &tmap_kv, fb, c * 64, g, pageA * kPage, pol_kv);
+            if (npg == 2) tma_load_3d(dst + kPageChunkBytes, &tmap_kv, fb, c * 64, g, pageB * kPage, pol_kv);
+            issued[st.idx] = true;
+            issued_phase[st.idx] = st.phase;
+            st.next(kRing);
+          }
+        }
+        return true;
       });
       if (!ok) {  // drain copies still in flight before the CTA may exit
-        for (int s = 0; s < kStages; ++s)
-          if (issued[s]) mbar_wait_drain(bar(kBarFull + s), issued_phase[s]);
+        for (int s = 0; s < kRing; ++s)
+          if (issued[s]) mbar_wait_drain(bar(kBarRingFull + s), issued_phase[s]);
+        if (qr_issued) mbar_wait_drain(bar(kBarQrFull), qr_issued_phase);
       }
     } else if (warp == 1 && lane == 0) {
-      // ---- MMA issuer: S = Q K^T
+      // ---- MMA issuer: S = Q K^T for page pairs (N = 128) or a single page (N = 64)
       Ring st, sb;
-      uint32_t qphase = 0;
+      uint32_t q_phase = 0, qr_phase = 0;
       bool ok = true;
-      const uint32_t idesc = make_idesc_bf16(128, 64, 0, 0);
+      const uint32_t idesc128 = make_idesc_bf16(128, 128, 0, 0);
+      const uint32_t idesc64 = make_idesc_bf16(128, 64, 0, 0);
+      const uint64_t ring_desc0 = make_smem_desc(sbase + OFF_RING, 16, 1024, 2);
+      const uint64_t qr_desc = make_smem_desc(sbase + OFF_QROPE, 16, 1024, 2);
+      const uint32_t ring_empty0 = bar(kBarRingEmpty);
+      const uint32_t ring_full0 = bar(kBarRingFull);
       for_each_piece(P, it, [&](int, int p0, int p1, int) {
-        for (int p = p0; p < p1; ++p) {
-          ok = mbar_wait(bar(kBarFull + st.idx), st.phase, abortf, P.err, kErrWaitBase + 2) &&
-               mbar_wait(bar(kBarSFree + sb.idx), sb.phase ^ 1u, abortf, P.err, kErrWaitBase + 3);
-          if (ok && p == p0) {
-            ok = mbar_wait(bar(kBarQFull), qphase, abortf, P.err, kErrWaitBase + 4);
-            qphase ^= 1u;
+        st.advance(kRing, 8);  // query chunks are consumed by the softmax warps
+        bool first = true;
+        for (int pa = p0; pa < p1; pa += 2) {
+          const int npg = (pa + 1 < p1) ? 2 : 1;
+          const uint32_t idesc = npg == 2 ? idesc128 : idesc64;
+          const bool last_pair = pa + 2 >= p1;
+          ok = mbar_wait(bar(kBarSFree + sb.idx), sb.phase ^ 1u, abortf, P.err, kErrWaitBase + 4);
+          if (ok && first) {
+            ok = mbar_wait(bar(kBarQFull), q_phase, abortf, P.err, kErrWaitBase + 5);
+            q_phase ^= 1u;
           }
           if (!ok) return false;
+          const uint32_t dS = tmem + kTmemS + 128u * sb.idx;
+          // the pair's 9 chunk stages, issued fully unrolled with precomputed
+          // stage indices: per-chunk waits stay (TMA streams chunk by chunk) but
+          // no descriptor or ring arithmetic sits between the MMAs
           tc_fence_after();
-          const uint32_t kst = sbase + st.idx * kKStageBytes;
-          const uint32_t dS = tmem + kTmemS + 64u * sb.idx;
-#pragma unroll 4
-          for (int s = 0; s < 36; ++s) {
-            const uint64_t bdesc =
-                make_smem_desc(kst + (s >> 2) * kChunkBytes + (s & 3) * 32, 16, 1024, 2);
-            mma_ts(dS, tmem + kTmemQ + 8u * s, bdesc, idesc, s > 0);
+          uint32_t sidx[9], sph[9];
+#pragma unroll
+          for (int c = 0; c < 9; ++c) {
+            sidx[c] = st.idx;
+            sph[c] = st.phase;
+            st.next(kRing);
           }
-          tc_commit(bar(kBarEmpty + st.idx));
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            if (!mbar_wait(ring_full0 + 8u * sidx[c], sph[c], abortf, P.err, kErrWaitBase + 6))
+              return false;
+            const uint64_t bd = ring_desc0 + (uint64_t)(sidx[c] * (kChunkBytes >> 4));
+            const uint32_t a = tmem + kTmemQ + 32u * c;
+            mma_ts(dS, a, bd, idesc, c > 0);
+            mma_ts(dS, a + 8, bd + 2, idesc, 1);
+            mma_ts(dS, a + 16, bd + 4, idesc, 1);
+            mma_ts(dS, a + 24, bd + 6, idesc, 1);
+            tc_commit(ring_empty0 + 8u * sidx[c]);
+          }
+          if (!mbar_wait(ring_full0 + 8u * sidx[8], sph[8], abortf, P.err, kErrWaitBase + 7))
+            return false;
+          if (first) {
+            if (!mbar_wait(bar(kBarQrFull), qr_phase, abortf, P.err, kErrWaitBase + 8)) return false;
+            qr_phase ^= 1u;
+          }
+          {
+            const uint64_t bd = ring_desc0 + (uint64_t)(sidx[8] * (kChunkBytes >> 4));
+            mma_ss(dS, qr_desc, bd, idesc, 1);
+            mma_ss(dS, qr_desc + 2, bd + 2, idesc, 1);
+            mma_ss(dS, qr_desc + 4, bd + 4, idesc, 1);
+            mma_ss(dS, qr_desc + 6, bd + 6, idesc, 1);
+            tc_commit(ring_empty0 + 8u * sidx[8]);
+          }
           tc_commit(bar(kBarSFull + sb.idx));
-          st.next(kStages);
+          if (last_pair) tc_commit(bar(kBarQrEmpty));
           sb.next(2);
+          first = false;
         }
         return true;
       });
       tc_commit(bar(kBarDrain));
       mbar_wait_drain(bar(kBarDrain), 0);
     } else if (warp >= 4) {
-      // ---- softmax warpgroup: thread r owns query row r of the tile
-      const int r = tid - 128;
+      // ---- two softmax warpgroups: thread (wg, r) owns query row r; of each page
+      // pair, warpgroup 0 handles the first page and warpgroup 1 the second
+      const int wg = (tid - 128) >> 7;
+      const int r = (tid - 128) & 127;
+      const uint32_t bar_wg = 1u + (uint32_t)wg;  // named barrier of this warpgroup (128)
+      const uint32_t bar_all = 3u;                // named barrier of both groups (256)
       const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
       const int rr = rg * kRows + r;
       const bool valid = rr < P.R;
       const int qi = valid ? rr / P.hpk : 0;
       const int head = valid ? g * P.hpk + rr % P.hpk : 0;
       const float c = P.scale_log2;
-      const float kTau = 8.0f;
-      Ring sb, ps;
+      float* xmax = reinterpret_cast<float*>(smem + OFF_XCH);  // [2 pair parities][2 groups][128]
+      float* xl = xmax + 4 * kRows;                            // [2][128] exact row sums
+      float* xlr = xl + 2 * kRows;                             // [2][128] rounded row sums
+      Ring st, sb;
+      uint32_t kp = 0;    // running page index of this cluster (P slot = kp % 4)
+      uint32_t npair = 0; // running pair index (exchange-buffer parity)
       bool ok = true;
+      const uint32_t p_remote = map_to_rank(sbase + OFF_P, peer);
+      const uint32_t side_remote = map_to_rank(smem_u32(side), peer);
+      const uint32_t pfull_remote = map_to_rank(bar(kBarPFull), peer);
+      const uint32_t prow_off = (uint32_t)((r >> 3) * 1024 + (r & 7) * 128);
+      // Every bounded wait is followed by an AND over all 256 threads, so both
+      // groups always leave together (named barriers have no timeout).
       for_each_piece(P, it, [&](int b, int p0, int p1, int ordinal) {
         const int L = max(P.seqlens[b], 0);
         const int limit = valid ? (P.causal ? L - P.s_q + qi : L - 1) : -1;
-        // Q row -> TMEM columns [0, 288) as packed bf16 pairs
+        // latent query chunks -> TMEM columns [32c, 32c + 32): group 0 copies
+        // chunks 0-3, group 1 chunks 4-7
         {
-          const uint4* src = reinterpret_cast<const uint4*>(
-              P.q + ((size_t)(b * P.s_q + qi) * P.h_q + head) * kD);
-#pragma unroll 1
-          for (int j = 0; j < 9; ++j) {
+          Ring q = st;
+          q.advance(kRing, 4u * (uint32_t)wg);
+          for (int cc = 4 * wg; cc < 4 * wg + 4; ++cc) {
+            ok = named_bar_and(bar_all, 256, mbar_wait(bar(kBarRingFull + q.idx), q.phase, abortf, P.err,
+                                                       kErrWaitBase + 9));
+            if (!ok) return false;
+            const uint8_t* row = smem + OFF_RING + q.idx * kChunkBytes + r * 128;
             uint32_t v[32];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-              uint4 x = valid ? __ldg(src + 8 * j + u) : make_uint4(0, 0, 0, 0);
+              const uint4 x = *reinterpret_cast<const uint4*>(row + ((u ^ (r & 7)) << 4));
               v[4 * u] = x.x; v[4 * u + 1] = x.y; v[4 * u + 2] = x.z; v[4 * u + 3] = x.w;
             }
-            tmem_st32(tmem + lane_off + kTmemQ + 32 * j, v);
+            tmem_st32(tmem + lane_off + kTmemQ + 32u * cc, v);
+            named_bar_sync(bar_wg, 128);
+            if (r == 0) mbar_arrive(bar(kBarRingEmpty + q.idx));
+            q.next(kRing);
           }
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(bar(kBarQFull));
         }
-        // l: exact row sum (for lse); lr: sum of the bf16-rounded weights the
-        // MMA multiplies (normalises O so the applied weights sum to one)
+        st.advance(kRing, 8u + 9u * (uint32_t)((p1 - p0 + 1) / 2));  // page chunks: MMA thread's
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(kBarQFull));
+
+        // this group's share of the row sums: l exact (for lse), lr of the
+        // bf16-rounded weights the MMA multiplies (normalises O)
         float m_ref = -INFINITY, l = 0.f, lr = 0.f;
-        for (int p = p0; p < p1; ++p) {
-          // every bounded wait is followed by a group-wide AND so that all 128
-          // threads leave together (a named barrier has no timeout)
-          ok = named_bar_and(1, 128,
-                             mbar_wait(bar(kBarSFull + sb.idx), sb.phase, abortf, P.err, kErrWaitBase + 5));
+        for (int pa = p0; pa < p1; pa += 2, ++npair) {
+          const int npg = (pa + 1 < p1) ? 2 : 1;
+          const bool last_pair = pa + 2 >= p1;
+          const bool mine = wg < npg;  // uniform per group
+          ok = named_bar_and(bar_all, 256, mbar_wait(bar(kBarSFull + sb.idx), sb.phase, abortf, P.err,
+                                                     kErrWaitBase + 10));
           if (!ok) return false;
           tc_fence_after();
-          uint32_t sa[32], sbv[32];
-          tmem_ld64_sync(tmem + lane_off + kTmemS + 64u * sb.idx, sa, sbv);
+          const int jw = (pa + wg) * kPage;  // first token of this group's page
+          uint32_t s0[32], s1[32];
+          if (mine) {
+            tmem_ld64_sync(tmem + lane_off + kTmemS + 128u * sb.idx + 64u * (uint32_t)wg, s0, s1);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) { s0[j] = 0xff800000u; s1[j] = 0xff800000u; }  // -inf
+          }
           tc_fence_before();
           mbar_arrive(bar(kBarSFree + sb.idx));
           sb.next(2);
-          float s[64];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            s[j] = __uint_as_float(sa[j]);
-            s[32 + j] = __uint_as_float(sbv[j]);
-          }
-          // tokens past the row's last visible index get weight 0; only the
-          // tail page(s) of a sequence carry such tokens
-          const int j0 = p * kPage;
-          const bool tail = j0 + kPage - 1 > limit;
+          const bool tail = mine && (jw + kPage - 1 > limit);
           if (tail) {
 #pragma unroll
-            for (int j = 0; j < 64; ++j)
-              if (j0 + j > limit) s[j] = -INFINITY;
+            for (int j = 0; j < 32; ++j) {
+              if (jw + j > limit) s0[j] = 0xff800000u;
+              if (jw + 32 + j > limit) s1[j] = 0xff800000u;
+            }
           }
-          float mx = s[0];
+          float mloc;
+          {
+            float m8[8];
 #pragma unroll
-          for (int j = 1; j < 64; ++j) mx = fmaxf(mx, s[j]);
+            for (int u = 0; u < 8; ++u) m8[u] = fmaxf(__uint_as_float(s0[u]), __uint_as_float(s1[u]));
+#pragma unroll
+            for (int j = 8; j < 32; ++j)
+              m8[j & 7] = fmaxf(m8[j & 7], fmaxf(__uint_as_float(s0[j]), __uint_as_float(s1[j])));
+            mloc = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                         fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          }
+          // exchange the row max with the other group (buffer alternates by pair)
+          float* xm = xmax + (npair & 1u) * (2 * kRows);
+          xm[wg * kRows + r] = mloc;
+          named_bar_sync(bar_all, 256);
+          const float mx = fmaxf(mloc, xm[(wg ^ 1) * kRows + r]);
+          // identical lazy-rescale update in both groups
           const float mxs = (mx == -INFINITY) ? -INFINITY : mx * c;
           float alpha = 1.f;
           bool resc = false;
@@ -341,52 +529,81 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const DecodeParams P)
             m_ref = mxs;
           }
           const float base = (m_ref == -INFINITY) ? 0.f : m_ref;
-          uint32_t pk[32];
-          float lsum = 0.f, lrsum = 0.f;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            float e0 = ex2(fmaf(s[2 * j], c, -base));
-            float e1 = ex2(fmaf(s[2 * j + 1], c, -base));
-            if (tail) {
-              e0 = (j0 + 2 * j > limit) ? 0.f : e0;
-              e1 = (j0 + 2 * j + 1 > limit) ? 0.f : e1;
-            }
-            pk[j] = pack_bf16x2(e0, e1);
-            lsum += e0 + e1;
-            lrsum += __uint_as_float(pk[j] << 16) + __uint_as_float(pk[j] & 0xffff0000u);
-          }
-          l += lsum;
-          lr += lrsum;
-          const bool last = (p == p1 - 1);
-          // wait until the O-CTA's MMAs have finished reading this P slot
-          ok = named_bar_and(1, 128, mbar_wait<true>(bar(kBarPFree + ps.idx), ps.phase ^ 1u, abortf,
-                                                      P.err, kErrWaitBase + 6));
+          const uint32_t wany = __any_sync(0xffffffffu, resc) ? 1u : 0u;
+          const uint32_t kk = kp + (uint32_t)wg;
+          const uint32_t slot = kk % kPSlots, buf = kk % kStageBufs;
+          // the destination slot must be consumed and the staging buffer copied out
+          bool got = true;
+          if (mine)
+            got = mbar_wait<true>(bar(kBarPFree + slot), ((kk / kPSlots) & 1u) ^ 1u, abortf, P.err,
+                                  kErrWaitBase + 11) &&
+                  mbar_wait<true>(bar(kBarStageFree + buf), ((kk / kStageBufs) & 1u) ^ 1u, abortf,
+                                  P.err, kErrWaitBase + 21);
+          ok = named_bar_and(bar_all, 256, got);
           if (!ok) return false;
-          const uint32_t prow = sbase + OFF_P + ps.idx * kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
+          uint32_t pk[32];
+          if (mine) {
+            // P = exp2(S*c - base) -> bf16; masked entries are -inf and weigh exactly 0
+            float ls[4] = {0.f, 0.f, 0.f, 0.f}, lrs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc)
-            st_cluster_v4(map_to_rank(prow + ((cc ^ (r & 7)) << 4), peer), pk[4 * cc],
-                          pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-          const uint32_t side_local = smem_u32(&side[ps.idx]);
-          st_cluster_f32(map_to_rank(side_local + offsetof(SideSlot, alpha) + 4 * r, peer), alpha);
-          if (last)
-            st_cluster_f32(map_to_rank(side_local + offsetof(SideSlot, linv) + 4 * r, peer),
-                           lr > 0.f ? 1.f / lr : 0.f);
-          fence_proxy_async_cluster();
-          const bool any = named_bar_or(1, 128, resc);
-          if (r == 0) {
-            st_cluster_u32(map_to_rank(side_local, peer), (any ? 1u : 0u) | (last ? 2u : 0u));
-            mbar_arrive_remote(map_to_rank(bar(kBarPFull + ps.idx), peer));
+            for (int j = 0; j < 16; ++j) {
+              float e0 = ex2(fmaf(__uint_as_float(s0[2 * j]), c, -base));
+              float e1 = ex2(fmaf(__uint_as_float(s0[2 * j + 1]), c, -base));
+              float e2 = ex2(fmaf(__uint_as_float(s1[2 * j]), c, -base));
+              float e3 = ex2(fmaf(__uint_as_float(s1[2 * j + 1]), c, -base));
+              if (tail) {  // also exact when c == 0
+                e0 = s0[2 * j] == 0xff800000u ? 0.f : e0;
+                e1 = s0[2 * j + 1] == 0xff800000u ? 0.f : e1;
+                e2 = s1[2 * j] == 0xff800000u ? 0.f : e2;
+                e3 = s1[2 * j + 1] == 0xff800000u ? 0.f : e3;
+              }
+              pk[j] = pack_bf16x2(e0, e1);
+              pk[16 + j] = pack_bf16x2(e2, e3);
+              ls[j & 3] += (e0 + e1) + (e2 + e3);
+              lrs[j & 3] += (__uint_as_float(pk[j] << 16) + __uint_as_float(pk[j] & 0xffff0000u)) +
+                            (__uint_as_float(pk[16 + j] << 16) + __uint_as_float(pk[16 + j] & 0xffff0000u));
+            }
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            lr += (lrs[0] + lrs[1]) + (lrs[2] + lrs[3]);
           }
-          ps.next(2);
-        }
-        if (valid) {
-          const float lse_v = l > 0.f ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-          const int slot = piece_slot(P, b, ordinal);
-          if (slot < 0)
-            P.lse[((size_t)b * P.h_q + head) * P.s_q + qi] = lse_v;
-          else
-            P.part_lse[((size_t)slot * P.h_kv + g) * P.R + rr] = lse_v;
+          float ltot = 0.f, lrtot = 0.f;
+          if (last_pair) {  // the piece's totals: both groups' shares
+            xl[wg * kRows + r] = l;
+            xlr[wg * kRows + r] = lr;
+            named_bar_sync(bar_all, 256);
+            ltot = l + xl[(wg ^ 1) * kRows + r];
+            lrtot = lr + xlr[(wg ^ 1) * kRows + r];
+          }
+          if (mine) {
+            // P row and the row's factors into the local staging buffers, then
+            // one bulk copy each into the O-CTA's slot
+            uint8_t* srow = smem + OFF_STAGE + buf * kPBytes + prow_off;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<uint4*>(srow + ((q ^ (r & 7)) << 4)) =
+                  make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+            SideSlot* ss = reinterpret_cast<SideSlot*>(smem + OFF_STAGE_SIDE + buf * kSideBytes);
+            ss->alpha[r] = wg == 0 ? alpha : 1.f;
+            ss->linv[r] = lrtot > 0.f ? 1.f / lrtot : 0.f;
+            if (lane == 0) ss->wflag[warp & 3] = wg == 0 ? wany : 0u;
+            fence_proxy_async_cta();  // staged data is read by the bulk copies (async proxy)
+            named_bar_sync(bar_wg, 128);
+            if (r == 0) {
+              const uint32_t rbar = pfull_remote + slot * 8u;
+              bulk_copy_to_peer(p_remote + slot * kPBytes, sbase + OFF_STAGE + buf * kPBytes, kPBytes, rbar);
+              bulk_copy_to_peer(side_remote + slot * kSideBytes, sbase + OFF_STAGE_SIDE + buf * kSideBytes,
+                                kSideBytes, rbar);
+            }
+          }
+          kp += (uint32_t)npg;
+          if (last_pair && valid && wg == 0) {
+            const float lse_v = ltot > 0.f ? (m_ref + __log2f(ltot)) * kLn2 : -INFINITY;
+            const int pslot = piece_slot(P, b, ordinal);
+            if (pslot < 0)
+              P.lse[((size_t)b * P.h_q + head) * P.s_q + qi] = lse_v;
+            else
+              P.part_lse[((size_t)pslot * P.h_kv + g) * P.R + rr] = lse_v;
+          }
         }
         return true;
       });
@@ -394,124 +611,150 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const DecodeParams P)
   } else {
     // =========================================================== O-CTA
     if (warp == 0 && lane == 0) {
-      // ---- TMA producer: value part of each page (8 chunks)
+      // ---- TMA producer: value part of each page as two half-page stages
       Ring st;
       bool ok = true;
-      uint32_t issued_phase[kStages];
-      bool issued[kStages] = {false, false, false};
+      uint32_t issued_phase[kVStages];
+      bool issued[kVStages] = {false, false, false, false};
       const uint64_t pol = policy_evict_first();
       for_each_piece(P, it, [&](int b, int p0, int p1, int) {
         for (int p = p0; p < p1 && ok; ++p) {
-          ok = mbar_wait(bar(kBarEmpty + st.idx), st.phase ^ 1u, abortf, P.err, kErrWaitBase + 11);
-          if (!ok) break;
-          int page = P.block_table[(size_t)b * P.max_pages + p];
-          if (page < 0 || page >= P.num_pages) page = P.num_pages;
-          const uint32_t fb = bar(kBarFull + st.idx);
-          mbar_arrive_expect_tx(fb, kVStageBytes);
-          const uint32_t dst = sbase + st.idx * kVStageBytes;
+          const int page = load_page(P, b, p);
+          for (int hh = 0; hh < 2 && ok; ++hh) {
+            ok = mbar_wait(bar(kBarVEmpty + st.idx), st.phase ^ 1u, abortf, P.err, kErrWaitBase + 12);
+            if (!ok) break;
+            const uint32_t fb = bar(kBarVFull + st.idx);
+            mbar_arrive_expect_tx(fb, kVStageBytes);
+            const uint32_t dst = sbase + OFF_V + st.idx * kVStageBytes;
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc)
-            tma_load_3d(dst + cc * kChunkBytes, &tmap_kv, fb, cc * 64, g, page * kPage, pol);
-          issued[st.idx] = true;
-          issued_phase[st.idx] = st.phase;
-          st.next(kStages);
+            for (int j = 0; j < 4; ++j)
+              tma_load_3d(dst + j * kPageChunkBytes, &tmap_kv, fb, (4 * hh + j) * 64, g, page * kPage, pol);
+            issued[st.idx] = true;
+            issued_phase[st.idx] = st.phase;
+            st.next(kVStages);
+          }
         }
         return ok;
       });
       if (!ok) {
-        for (int s = 0; s < kStages; ++s)
-          if (issued[s]) mbar_wait_drain(bar(kBarFull + s), issued_phase[s]);
+        for (int s = 0; s < kVStages; ++s)
+          if (issued[s]) mbar_wait_drain(bar(kBarVFull + s), issued_phase[s]);
       }
     } else if (warp == 1 && lane == 0) {
       // ---- MMA issuer: O += P V, plus the command stream to the correction warps
-      Ring st, ps;
-      uint32_t done_phase = 0, drain_phase = 0;
+      Ring st;
+      uint32_t kp = 0, done_phase = 0, drain_phase = 0;
       bool pending_epilogue = false, ok = true;
       const uint32_t idesc = make_idesc_bf16(128, 256, 0, 1);
+      const uint64_t v_desc0 = make_smem_desc(sbase + OFF_V, 8192, 1024, 2);
+      const uint64_t p_desc0 = make_smem_desc(sbase + OFF_P, 16, 1024, 2);
       for_each_piece(P, it, [&](int b, int p0, int p1, int ordinal) {
-        for (int p = p0; p < p1; ++p) {
-          ok = mbar_wait(bar(kBarFull + st.idx), st.phase, abortf, P.err, kErrWaitBase + 12) &&
-               mbar_wait<true>(bar(kBarPFull + ps.idx), ps.phase, abortf, P.err,
-                               kErrWaitBase + 13);
-          if (!ok) return false;
-          const uint32_t flags = *reinterpret_cast<volatile uint32_t*>(&side[ps.idx].flags);
-          const bool first = (p == p0);
+        for (int p = p0; p < p1; ++p, ++kp) {
+          const uint32_t ps = kp % kPSlots, pph = (kp / kPSlots) & 1u;
+          if (!mbar_wait<true>(bar(kBarPFull + ps), pph, abortf, P.err, kErrWaitBase + 13)) return false;
+          const volatile uint32_t* wf = side[ps].wflag;
+          const bool resc = (wf[0] | wf[1] | wf[2] | wf[3]) != 0u;
+          const bool first = (p == p0), last = (p == p1 - 1);
           if (first && pending_epilogue) {  // accumulator still being drained by the epilogue
             ok = mbar_wait(bar(kBarCmdDone), done_phase, abortf, P.err, kErrWaitBase + 14);
             done_phase ^= 1u;
             pending_epilogue = false;
             if (!ok) return false;
           }
-          if ((flags & 1u) && !first) {
+          if (last) {  // keep this piece's 1/l: the side slot is recycled soon after
+            const float4* srcl = reinterpret_cast<const float4*>(side[ps].linv);
+            float4* dstl = reinterpret_cast<float4*>(mail->linv);
+#pragma unroll 4
+            for (int u = 0; u < kRows / 4; ++u) dstl[u] = srcl[u];
+          }
+          if (resc && !first) {
             // a row's reference max moved: finish all issued MMAs, rescale O rows
             tc_commit(bar(kBarDrain));
             ok = mbar_wait(bar(kBarDrain), drain_phase, abortf, P.err, kErrWaitBase + 15);
             drain_phase ^= 1u;
             if (!ok) return false;
             mail->cmd = kCmdRescale;
-            mail->slot = ps.idx;
+            mail->slot = (int)ps;
             tc_fence_before();
-            mbar_arrive(bar(kBarQFull));
+            mbar_arrive(bar(kBarCmdFull));
             ok = mbar_wait(bar(kBarCmdDone), done_phase, abortf, P.err, kErrWaitBase + 16);
             done_phase ^= 1u;
             if (!ok) return false;
           }
+          const uint64_t pd = p_desc0 + (uint64_t)(ps * (kPBytes >> 4));
+          uint32_t vidx[2];
+#pragma unroll
+          for (int n = 0; n < 2; ++n) {
+            vidx[n] = st.idx;
+            if (!mbar_wait(bar(kBarVFull + st.idx), st.phase, abortf, P.err, kErrWaitBase + 17))
+              return false;
+            st.next(kVStages);
+          }
           tc_fence_after();
-          const uint32_t vst = sbase + st.idx * kVStageBytes;
-          const uint32_t pslot = sbase + OFF_P + ps.idx * kPBytes;
 #pragma unroll
-          for (int n = 0; n < 2; ++n)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t adesc = make_smem_desc(pslot + k * 32, 16, 1024, 2);
-              const uint64_t bdesc =
-                  make_smem_desc(vst + (4 * n) * kChunkBytes + k * 2048, 8192, 1024, 2);
-              mma_ss(tmem + kTmemO + 256u * n, adesc, bdesc, idesc, !(first && k == 0));
-            }
-          tc_commit(bar(kBarEmpty + st.idx));
-          tc_commit(bar(kBarSFull + ps.idx));  // P slot consumed -> relay warp
-          if (flags & 2u) {
+          for (int n = 0; n < 2; ++n) {
+            const uint64_t vd = v_desc0 + (uint64_t)(vidx[n] * (kVStageBytes >> 4));
+            const uint32_t d = tmem + kTmemO + 256u * n;
+            mma_ss(d, pd, vd, idesc, !first);
+            mma_ss(d, pd + 2, vd + 128, idesc, 1);
+            mma_ss(d, pd + 4, vd + 256, idesc, 1);
+            mma_ss(d, pd + 6, vd + 384, idesc, 1);
+            tc_commit(bar(kBarVEmpty + vidx[n]));
+          }
+          tc_commit(bar(kBarPCons + ps));  // P slot consumed -> relay warp
+          if (last) {
             // last page of the piece: wait for the accumulator, hand it to the epilogue
             tc_commit(bar(kBarDrain));
-            ok = mbar_wait(bar(kBarDrain), drain_phase, abortf, P.err, kErrWaitBase + 17);
+            ok = mbar_wait(bar(kBarDrain), drain_phase, abortf, P.err, kErrWaitBase + 18);
             drain_phase ^= 1u;
             if (!ok) return false;
-            const float4* srcl = reinterpret_cast<const float4*>(side[ps.idx].linv);
-            float4* dstl = reinterpret_cast<float4*>(mail->linv);
-#pragma unroll 4
-            for (int u = 0; u < kRows / 4; ++u) dstl[u] = srcl[u];
             mail->cmd = kCmdEpilogue;
             mail->b = b;
             mail->part_slot = piece_slot(P, b, ordinal);
             tc_fence_before();
-            mbar_arrive(bar(kBarQFull));
+            mbar_arrive(bar(kBarCmdFull));
             pending_epilogue = true;
           }
-          st.next(kStages);
-          ps.next(2);
         }
         return true;
       });
-      if (pending_epilogue)
-        mbar_wait(bar(kBarCmdDone), done_phase, abortf, nullptr, 0);
+      if (pending_epilogue) mbar_wait(bar(kBarCmdDone), done_phase, abortf, nullptr, 0);
       tc_commit(bar(kBarDrain));
       mbar_wait_drain(bar(kBarDrain), drain_phase);
     } else if (warp == 2 && lane == 0) {
-      // ---- relay: tell the S-CTA a P slot may be overwritten once its MMAs completed
-      Ring ps;
+      // ---- relay: re-arm a consumed P slot and hand it back to the S-CTA
+      uint32_t kp = 0;
+      const uint32_t pfree_remote = map_to_rank(bar(kBarPFree), peer);
       for_each_piece(P, it, [&](int, int p0, int p1, int) {
-        for (int p = p0; p < p1; ++p) {
-          if (!mbar_wait(bar(kBarSFull + ps.idx), ps.phase, abortf, P.err, kErrWaitBase + 18))
+        for (int p = p0; p < p1; ++p, ++kp) {
+          const uint32_t ps = kp % kPSlots, pph = (kp / kPSlots) & 1u;
+          if (!mbar_wait(bar(kBarPCons + ps), pph, abortf, P.err, kErrWaitBase + 19)) return false;
+          mbar_arrive_expect_tx(bar(kBarPFull + ps), kPFullTx);
+          mbar_arrive_remote(pfree_remote + ps * 8u);
+        }
+        return true;
+      });
+    } else if (warp == 3 && lane == 0) {
+      // ---- land relay: once a P message has landed, its staging buffer in the
+      // S-CTA may be reused
+      uint32_t kp = 0;
+      const uint32_t sfree_remote = map_to_rank(bar(kBarStageFree), peer);
+      for_each_piece(P, it, [&](int, int p0, int p1, int) {
+        for (int p = p0; p < p1; ++p, ++kp) {
+          if (!mbar_wait<true>(bar(kBarPFull + kp % kPSlots), (kp / kPSlots) & 1u, abortf, P.err,
+                               kErrWaitBase + 22))
             return false;
-          mbar_arrive_remote(map_to_rank(bar(kBarPFree + ps.idx), peer));
-          ps.next(2);
+          mbar_arrive_remote(sfree_remote + (kp % kStageBufs) * 8u);
         }
         return true;
       });
     } else if (warp >= 4) {
-      // ---- correction / epilogue warpgroup: thread r owns TMEM lane r (= row r)
-      const int r = tid - 128;
+      // ---- two correction / epilogue warpgroups: thread (wg, r) owns TMEM lane
+      // r (= row r) and accumulator columns [256 wg, 256 wg + 256)
+      const int wg = (tid - 128) >> 7;
+      const int r = (tid - 128) & 127;
       const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+      const uint32_t tcol = tmem + lane_off + kTmemO + 256u * (uint32_t)wg;
       const int rr = rg * kRows + r;
       const bool valid = rr < P.R;
       const int qi = valid ? rr / P.hpk : 0;
@@ -520,7 +763,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const DecodeParams P)
       for_each_piece(P, it, [&](int, int, int, int) {
         for (;;) {
           if (!__all_sync(0xffffffffu,
-                          mbar_wait(bar(kBarQFull), cmd_phase, abortf, P.err, kErrWaitBase + 19)))
+                          mbar_wait(bar(kBarCmdFull), cmd_phase, abortf, P.err, kErrWaitBase + 20)))
             return false;
           cmd_phase ^= 1u;
           tc_fence_after();
@@ -529,12 +772,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const DecodeParams P)
             const float a = side[mail->slot].alpha[r];
             if (__any_sync(0xffffffffu, a != 1.f)) {  // tcgen05.ld/st are warp-collective
 #pragma unroll 1
-              for (int j = 0; j < 16; ++j) {
+              for (int j = 0; j < 8; ++j) {
                 uint32_t v[32];
-                tmem_ld32_sync(tmem + lane_off + kTmemO + 32 * j, v);
+                tmem_ld32_sync(tcol + 32 * j, v);
 #pragma unroll
                 for (int u = 0; u < 32; ++u) v[u] = __float_as_uint(__uint_as_float(v[u]) * a);
-                tmem_st32(tmem + lane_off + kTmemO + 32 * j, v);
+                tmem_st32(tcol + 32 * j, v);
               }
               tmem_wait_st();
             }
@@ -542,43 +785,44 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const DecodeParams P)
             mbar_arrive(bar(kBarCmdDone));
             continue;
           }
-          // epilogue
+          // epilogue: tcgen05.ld is warp-collective, so every thread loads and
+          // only valid rows store
           const float linv = mail->linv[r];
           const int b = mail->b;
           const int pslot = mail->part_slot;
-          // tcgen05.ld is warp-collective: every thread loads, valid rows store
           if (pslot < 0) {
-            uint4* dst = reinterpret_cast<uint4*>(
-                P.o + ((size_t)(b * P.s_q + qi) * P.h_q + head) * kDV);
+            uint16_t* dst = P.o + ((size_t)(b * P.s_q + qi) * P.h_q + head) * kDV + 256 * wg;
 #pragma unroll 1
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < 8; ++j) {
               uint32_t v[32];
-              tmem_ld32_sync(tmem + lane_off + kTmemO + 32 * j, v);
+              tmem_ld32_sync(tcol + 32 * j, v);
               uint32_t pk[16];
 #pragma unroll
               for (int u = 0; u < 16; ++u)
-                pk[u] = pack_bf16x2(__uint_as_float(v[2 * u]) * linv,
-                                    __uint_as_float(v[2 * u + 1]) * linv);
+                pk[u] = pack_bf16x2(__uint_as_float(v[2 * u]) * linv, __uint_as_float(v[2 * u + 1]) * linv);
               if (valid) {
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                  dst[4 * j + u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                st_global_v8(dst + 32 * j, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+                st_global_v8(dst + 32 * j + 16, pk[8], pk[9], pk[10], pk[11], pk[12], pk[13], pk[14], pk[15]);
               }
             }
           } else {
-            float4* dst = reinterpret_cast<float4*>(
-                P.part_o + (((size_t)pslot * P.h_kv + g) * P.R + rr) * kDV);
+            float* dst = P.part_o + (((size_t)pslot * P.h_kv + g) * P.R + rr) * kDV + 256 * wg;
 #pragma unroll 1
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < 8; ++j) {
               uint32_t v[32];
-              tmem_ld32_sync(tmem + lane_off + kTmemO + 32 * j, v);
+              tmem_ld32_sync(tcol + 32 * j, v);
               if (valid) {
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
-                  dst[8 * j + u] = make_float4(__uint_as_float(v[4 * u]) * linv,
-                                               __uint_as_float(v[4 * u + 1]) * linv,
-                                               __uint_as_float(v[4 * u + 2]) * linv,
-                                               __uint_as_float(v[4 * u + 3]) * linv);
+                for (int u = 0; u < 4; ++u)
+                  st_global_v8(dst + 32 * j + 8 * u,
+                               __float_as_uint(__uint_as_float(v[8 * u]) * linv),
+                               __float_as_uint(__uint_as_float(v[8 * u + 1]) * linv),
+                               __float_as_uint(__uint_as_float(v[8 * u + 2]) * linv),
+                               __float_as_uint(__uint_as_float(v[8 * u + 3]) * linv),
+                               __float_as_uint(__uint_as_float(v[8 * u + 4]) * linv),
+                               __float_as_uint(__uint_as_float(v[8 * u + 5]) * linv),
+                               __float_as_uint(__uint_as_float(v[8 * u + 6]) * linv),
+                               __float_as_uint(__uint_as_float(v[8 * u + 7]) * linv));
               }
             }
           }
@@ -636,9 +880,10 @@ int decode_max_active_clusters(int device, int* out) {
   return 0;
 }
 
-cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, cudaStream_t stream) {
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, const CUtensorMap& tmap_q,
+                          cudaStream_t stream) {
   const int clusters = p.num_parts * p.h_kv * p.n_rg;
-  decode_kernel<<<2 * clusters, kThreads, SMEM_BYTES, stream>>>(tmap_kv, p);
+  decode_kernel<<<2 * clusters, kThreads, SMEM_BYTES, stream>>>(tmap_kv, tmap_q, p);
   return cudaGetLastError();
 }
 

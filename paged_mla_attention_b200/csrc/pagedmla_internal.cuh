@@ -61,7 +61,8 @@ cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, in
                             int32_t* num_splits, cudaStream_t stream);
 cudaError_t decode_prepare(int device);  // one-time per-device kernel attributes
 int decode_max_active_clusters(int device, int* out);
-cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, const CUtensorMap& tmap_q,
+                          cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 size_t decode_smem_bytes();
 

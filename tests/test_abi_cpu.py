@@ -56,11 +56,12 @@ def _decode(lib, **kw):
 
 @pytest.mark.parametrize("kw,code", [
     (dict(d=575), -2), (dict(dv=256), -2), (dict(h_q=15, h_kv=2), -2),
+    (dict(h_q=96), -2), (dict(h_q=12, h_kv=3), -2), (dict(h_q=320), -2),
     (dict(batch=-1), -1), (dict(s_q=0), -1), (dict(num_pages=0), -1), (dict(parts=0), -1),
     (dict(scale=float("nan")), -1), (dict(scale=-1.0), -1),
     (dict(q=None), -1), (dict(lse=None), -1), (dict(splits=None), -1),
-    (dict(q=0x10001), -3), (dict(o=0x70008), -3), (dict(kv=0x20002), -3),
-    (dict(ws_bytes=16), -5), (dict(ws=None), -5), (dict(ws=0x90004), -5),
+    (dict(q=0x10001), -3), (dict(o=0x70008), -3), (dict(o=0x70010), -3), (dict(kv=0x20002), -3),
+    (dict(ws_bytes=16), -5), (dict(ws=None), -5), (dict(ws=0x90004), -5), (dict(ws=0x90010), -5),
 ])
 def test_decode_rejects_bad_arguments(lib, kw, code):
     assert _decode(lib, **kw) == code
