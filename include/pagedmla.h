@@ -87,8 +87,13 @@ PMLA_API int mla_get_metadata_sizes(int batch, int num_heads_per_head_k, int num
  *       of sequence m[0]; m[5..7] are 0.
  *   num_splits             int32 [batch+1], device, out: exclusive prefix sum
  *       of pieces per sequence (0 pieces: empty sequence, 1: unsplit).
- *   num_parts              from mla_get_metadata_sizes for the same shape.
- * Errors: INVALID_ARG, CUDA.
+ *   num_parts              from mla_get_metadata_sizes for the same shape
+ *                          (any value in [1, 2048] is accepted).
+ * Part boundaries are spaced evenly in cost, assuming every part but the first
+ * starts inside a sequence, and snapped so no piece is shorter than two pages;
+ * no part costs more than ceil((total + (num_parts-1)*3) / num_parts) + 5,
+ * where total sums pages + 3 over the non-empty sequences.
+ * Errors: INVALID_ARG (num_parts outside [1, 2048], null pointers), CUDA.
  */
 PMLA_API int mla_get_metadata(const int32_t* cache_seqlens, int batch, int num_heads_per_head_k,
                      int num_heads_k, int32_t* tile_scheduler_metadata, int num_parts,

@@ -155,7 +155,8 @@ int mla_get_metadata(const int32_t* cache_seqlens, int batch, int num_heads_per_
   if (rc) return rc;
   if (!tile_scheduler_metadata || !num_splits || (batch > 0 && !cache_seqlens))
     return fail(PMLA_ERR_INVALID_ARG, "null pointer argument");
-  if (num_parts < 1) return fail(PMLA_ERR_INVALID_ARG, "num_parts %d < 1", num_parts);
+  if (num_parts < 1 || num_parts > pmla::kMaxParts)
+    return fail(PMLA_ERR_INVALID_ARG, "num_parts %d outside [1, %d]", num_parts, pmla::kMaxParts);
   cudaError_t e = pmla::launch_metadata(cache_seqlens, batch, num_parts, tile_scheduler_metadata,
                                         num_splits, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e, "metadata kernel launch");
@@ -226,6 +227,24 @@ int mla_decode_with_kvcache(const uint16_t* q, const uint16_t* kvcache, const in
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)cr);
 
+  // kvcache once more as a 4-D tensor [64 columns] x [tokens] x [9 column chunks]
+  // x [h_kv heads] (the chunk stride, 128 bytes, is below the token stride): one
+  // box of 64 columns x 64 tokens x 4 chunks lands as 4 chunk-major 8 KB tiles,
+  // i.e. half of a page's value part in a single TMA instruction.
+  CUtensorMap tmap_v;
+  {
+    cuuint64_t vdim[4] = {64, (cuuint64_t)num_pages * pmla::kPage, (cuuint64_t)pmla::kD / 64,
+                          (cuuint64_t)h_kv};
+    cuuint64_t vstride[3] = {(cuuint64_t)h_kv * pmla::kD * 2, 128, (cuuint64_t)pmla::kD * 2};
+    cuuint32_t vbox[4] = {64, (cuuint32_t)pmla::kPage, 4, 1};
+    cuuint32_t vestride[4] = {1, 1, 1, 1};
+    cr = encode(&tmap_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t*>(kvcache), vdim,
+                vstride, vbox, vestride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS)
+      return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled (value tiles) failed (%d)", (int)cr);
+  }
+
   // q as a 2-D tensor: [576 columns] x [batch*s_q*h_q rows]; boxes of 64 columns
   // x min(h_q/h_kv, 128) rows with the 128-byte swizzle.
   CUtensorMap tmap_q;
@@ -271,7 +290,7 @@ int mla_decode_with_kvcache(const uint16_t* q, const uint16_t* kvcache, const in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = pmla::decode_prepare(dev);
   if (e != cudaSuccess) return fail_cuda(e, "decode kernel attributes");
-  e = pmla::launch_decode(p, tmap, tmap_q, st);
+  e = pmla::launch_decode(p, tmap, tmap_q, tmap_v, st);
   if (e != cudaSuccess) return fail_cuda(e, "decode kernel launch");
 
   pmla::CombineParams c;

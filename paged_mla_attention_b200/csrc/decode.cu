@@ -49,19 +49,18 @@ namespace pmla {
 namespace {
 
 constexpr int kThreads = 384;  // 4 role warps + two 4-warp groups
-constexpr int kRing = 10;                          // S-CTA chunk stages
-constexpr int kStageBufs = 2;                      // S-CTA P staging buffers
+constexpr int kRing = 8;                           // S-CTA chunk stages
+constexpr int kStageBufs = 4;                      // S-CTA P staging buffers
 constexpr uint32_t kChunkBytes = 128 * 64 * 2;     // 128 rows x 64 columns bf16
 constexpr uint32_t kPageChunkBytes = 64 * 64 * 2;  // one page's 64 tokens x 64 columns
 constexpr int kVStages = 4;                        // O-CTA half-page stages
 constexpr uint32_t kVStageBytes = 4 * kPageChunkBytes;  // 64 tokens x 256 columns
-constexpr int kPSlots = 4;
+constexpr int kPSlots = 5;
 constexpr uint32_t kPBytes = kRows * kPage * 2;    // 128 x 64 bf16
 
 struct SideSlot {        // per-P-slot row data sent with every P tile
   uint32_t wflag[4];     // per softmax warp: some row of the warp moved its reference max
   float alpha[kRows];    // O row rescale factors (1 = unchanged)
-  float linv[kRows];     // 1 / (sum of rounded weights) so far; used on a piece's last page
 };
 constexpr uint32_t kSideBytes = sizeof(SideSlot);
 constexpr uint32_t kPFullTx = kPBytes + kSideBytes;  // bytes every P message carries
@@ -71,27 +70,26 @@ struct Mailbox {         // MMA thread -> correction warps (O-CTA)
   int slot;              // P slot whose alpha to apply (rescale)
   int b;
   int part_slot;         // partial slot index, or -1 for a direct write
-  float linv[kRows];
+  float lr_x[2][2][kRows];  // [piece parity][correction group] row-sum halves
 };
 enum : int { kCmdRescale = 1, kCmdEpilogue = 2 };
 
 // mbarriers: one index space for both CTAs, each CTA initialises its own
 enum : int {
-  kBarRingFull = 0,                      // S [13] chunk stage loaded (TMA tx)
-  kBarRingEmpty = kBarRingFull + kRing,  // S [13] chunk stage consumed
+  kBarRingFull = 0,                      // S [kRing] chunk stage loaded (TMA tx)
+  kBarRingEmpty = kBarRingFull + kRing,  // S [kRing] chunk stage consumed
   kBarSFull = kBarRingEmpty + kRing,     // S [2] S tile ready (commit)
-  kBarSFree = kBarSFull + 2,             // S [2] S tile read by softmax warps (128)
-  kBarQFull = kBarSFree + 2,             // S Q latent in TMEM (128)
-  kBarQrFull = kBarQFull + 1,            // S Q RoPE chunk loaded (TMA tx)
+  kBarSFree = kBarSFull + 2,             // S [2] S tile read by softmax warps (256)
+  kBarQrFull = kBarSFree + 2,            // S Q RoPE chunk loaded (TMA tx)
   kBarQrEmpty = kBarQrFull + 1,          // S Q RoPE chunk no longer read (commit)
-  kBarPFree = kBarQrEmpty + 1,           // S [4] P slot free again (remote arrival)
-  kBarStageFree = kBarPFree + kPSlots,   // S [2] staging buffer copied out (remote arrival)
+  kBarPFree = kBarQrEmpty + 1,           // S [kPSlots] P slot free again (remote arrival)
+  kBarStageFree = kBarPFree + kPSlots,   // S [kStageBufs] staging buffer copied out (remote arrival)
   kBarVFull = kBarStageFree + kStageBufs,  // O [4] V half-stage loaded (TMA tx)
   kBarVEmpty = kBarVFull + kVStages,     // O [4] V half-stage consumed (commit)
-  kBarPFull = kBarVEmpty + kVStages,     // O [4] P slot written (armed + st.async tx)
-  kBarPCons = kBarPFull + kPSlots,       // O [4] P slot consumed (commit)
+  kBarPFull = kBarVEmpty + kVStages,     // O [kPSlots] P slot written (armed + bulk-copy tx)
+  kBarPCons = kBarPFull + kPSlots,       // O [kPSlots] P slot consumed (commit + 8 warps)
   kBarCmdFull = kBarPCons + kPSlots,     // O mailbox command posted (1)
-  kBarCmdDone = kBarCmdFull + 1,         // O command done (128)
+  kBarCmdDone = kBarCmdFull + 1,         // O command done (256)
   kBarDrain = kBarCmdDone + 1,           // both: all issued MMAs complete
   kNumBars = kBarDrain + 1
 };
@@ -112,8 +110,10 @@ constexpr uint32_t OFF_SIDE = OFF_P + kPSlots * kPBytes;          // O-CTA: side
 constexpr uint32_t OFF_MAIL = OFF_SIDE + kPSlots * kSideBytes;    // O-CTA: mailbox
 constexpr uint32_t OFF_STAGE_SIDE = OFF_STAGE + kStageBufs * kPBytes;  // S-CTA: staged side data
 constexpr uint32_t OFF_XCH = OFF_STAGE_SIDE + kStageBufs * kSideBytes;  // S-CTA: row exchange
-constexpr uint32_t kXchBytes = (2 * 2 * kRows + 2 * kRows + 2 * kRows) * 4;  // max x2 pairs, l, lr
-constexpr uint32_t OFF_CTRL = OFF_XCH + kXchBytes;                             // both
+constexpr uint32_t kXchBytes = (2 * 2 * kRows + 2 * kRows) * 4;  // max x2 pairs, l
+constexpr uint32_t cmax(uint32_t a, uint32_t b) { return a > b ? a : b; }
+constexpr uint32_t OFF_CTRL =  // both: after the larger of the two CTA layouts
+    (cmax(OFF_XCH + kXchBytes, OFF_MAIL + (uint32_t)sizeof(Mailbox)) + 15u) & ~15u;
 constexpr uint32_t SMEM_BYTES = OFF_CTRL + sizeof(Ctrl);
 static_assert(OFF_MAIL + sizeof(Mailbox) <= OFF_CTRL, "O-CTA regions overlap the control block");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget exceeded");
@@ -133,9 +133,6 @@ struct Ring {
   uint32_t idx = 0, phase = 0;
   __device__ __forceinline__ void next(uint32_t n) {
     if (++idx == n) { idx = 0; phase ^= 1u; }
-  }
-  __device__ __forceinline__ void advance(uint32_t n, uint32_t by) {
-    for (uint32_t i = 0; i < by; ++i) next(n);
   }
 };
 
@@ -206,6 +203,7 @@ __device__ __forceinline__ uint32_t load_q_chunk(const DecodeParams& P, const CU
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_q,
+              const __grid_constant__ CUtensorMap tmap_v,
               const DecodeParams P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -231,14 +229,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
   if (tid == 0) {
     if (rank == 0) {
       for (int s = 0; s < kRing; ++s) {
-        mbar_init(bar(kBarRingFull + s), 1);
+        mbar_init(bar(kBarRingFull + s), 2);  // one arrival per TMA producer
         mbar_init(bar(kBarRingEmpty + s), 1);
       }
       for (int s = 0; s < 2; ++s) {
         mbar_init(bar(kBarSFull + s), 1);
         mbar_init(bar(kBarSFree + s), 256);
       }
-      mbar_init(bar(kBarQFull), 256);
       mbar_init(bar(kBarQrFull), 1);
       mbar_init(bar(kBarQrEmpty), 1);
       for (int s = 0; s < kPSlots; ++s) mbar_init(bar(kBarPFree + s), 1);
@@ -250,7 +247,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
       }
       for (int s = 0; s < kPSlots; ++s) {
         mbar_init(bar(kBarPFull + s), 1);
-        mbar_init(bar(kBarPCons + s), 1);
+        mbar_init(bar(kBarPCons + s), 1 + 8);
       }
       mbar_init(bar(kBarCmdFull), 1);
       mbar_init(bar(kBarCmdDone), 256);
@@ -270,6 +267,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmap_kv);
     tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_v);
   }
   tc_fence_before();
   __syncthreads();
@@ -282,8 +280,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
 
   if (rank == 0) {
     // =========================================================== S-CTA
-    if (warp == 0 && lane == 0) {
-      // ---- TMA producer: query chunks, then chunk c of each page pair
+    if ((warp == 0 || warp == 2) && lane == 0) {
+      // ---- two TMA producers walk the same chunk-stage sequence; every stage's
+      // full barrier takes one arrival from each.  Producer 0 loads the query
+      // chunks and page A of each pair, producer 1 page B: one thread alone
+      // cannot issue 8 KB tiles fast enough to keep the SM's fill rate up.
+      const int prod = warp >> 1;
       Ring st;
       uint32_t qr_phase = 0;
       bool ok = true, qr_issued = false;
@@ -299,17 +301,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
           ok = mbar_wait(bar(kBarRingEmpty + st.idx), st.phase ^ 1u, abortf, P.err, kErrWaitBase + 1);
           if (!ok) return false;
           const uint32_t fb = bar(kBarRingFull + st.idx);
-          const uint32_t dst = sbase + OFF_RING + st.idx * kChunkBytes;
-          mbar_arrive_expect_tx(fb, load_q_chunk(P, &tmap_q, dst, fb, b, g, rg, c, pol_q, false));
-          load_q_chunk(P, &tmap_q, dst, fb, b, g, rg, c, pol_q, true);
-          issued[st.idx] = true;
-          issued_phase[st.idx] = st.phase;
+          if (prod == 0) {
+            const uint32_t dst = sbase + OFF_RING + st.idx * kChunkBytes;
+            mbar_arrive_expect_tx(fb, load_q_chunk(P, &tmap_q, dst, fb, b, g, rg, c, pol_q, false));
+            load_q_chunk(P, &tmap_q, dst, fb, b, g, rg, c, pol_q, true);
+            issued[st.idx] = true;
+            issued_phase[st.idx] = st.phase;
+          } else {
+            mbar_arrive(fb);
+          }
           st.next(kRing);
         }
         // RoPE chunk 8 into its own buffer (freed when the piece's MMAs are done)
-        ok = mbar_wait(bar(kBarQrEmpty), qr_phase ^ 1u, abortf, P.err, kErrWaitBase + 2);
-        if (!ok) return false;
-        {
+        if (prod == 0) {
+          ok = mbar_wait(bar(kBarQrEmpty), qr_phase ^ 1u, abortf, P.err, kErrWaitBase + 2);
+          if (!ok) return false;
           const uint32_t fb = bar(kBarQrFull);
           mbar_arrive_expect_tx(fb, load_q_chunk(P, &tmap_q, sbase + OFF_QROPE, fb, b, g, rg, 8, pol_q, false));
           load_q_chunk(P, &tmap_q, sbase + OFF_QROPE, fb, b, g, rg, 8, pol_q, true);
@@ -317,21 +323,24 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
           qr_issued_phase = qr_phase;
           qr_phase ^= 1u;
         }
-        // page pairs
+        // page pairs: chunk c of page A at +0, of page B at +8 KB
         for (int pa = p0; pa < p1; pa += 2) {
-          const int npg = (pa + 1 < p1) ? 2 : 1;
-          const int pageA = load_page(P, b, pa);
-          const int pageB = npg == 2 ? load_page(P, b, pa + 1) : 0;
+          const bool has = prod == 0 || pa + 1 < p1;
+          const int page = has ? load_page(P, b, pa + prod) : 0;
+          const uint32_t off = (uint32_t)prod * kPageChunkBytes;
           for (int c = 0; c < 9; ++c) {
             ok = mbar_wait(bar(kBarRingEmpty + st.idx), st.phase ^ 1u, abortf, P.err, kErrWaitBase + 3);
             if (!ok) return false;
             const uint32_t fb = bar(kBarRingFull + st.idx);
-            const uint32_t dst = sbase + OFF_RING + st.idx * kChunkBytes;
-            mbar_arrive_expect_tx(fb, (uint32_t)npg * kPageChunkBytes);
-            tma_load_3d(dst, &tmap_kv, fb, c * 64, g, pageA * kPage, pol_kv);
-            if (npg == 2) tma_load_3d(dst + kPageChunkBytes, &tmap_kv, fb, c * 64, g, pageB * kPage, pol_kv);
-            issued[st.idx] = true;
-            issued_phase[st.idx] = st.phase;
+            if (has) {
+              mbar_arrive_expect_tx(fb, kPageChunkBytes);
+              tma_load_3d(sbase + OFF_RING + st.idx * kChunkBytes + off, &tmap_kv, fb, c * 64, g,
+                          page * kPage, pol_kv);
+              issued[st.idx] = true;
+              issued_phase[st.idx] = st.phase;
+            } else {
+              mbar_arrive(fb);
+            }
             st.next(kRing);
           }
         }
@@ -345,7 +354,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
     } else if (warp == 1 && lane == 0) {
       // ---- MMA issuer: S = Q K^T for page pairs (N = 128) or a single page (N = 64)
       Ring st, sb;
-      uint32_t q_phase = 0, qr_phase = 0;
+      uint32_t qr_phase = 0;
       bool ok = true;
       const uint32_t idesc128 = make_idesc_bf16(128, 128, 0, 0);
       const uint32_t idesc64 = make_idesc_bf16(128, 64, 0, 0);
@@ -354,17 +363,25 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
       const uint32_t ring_empty0 = bar(kBarRingEmpty);
       const uint32_t ring_full0 = bar(kBarRingFull);
       for_each_piece(P, it, [&](int, int p0, int p1, int) {
-        st.advance(kRing, 8);  // query chunks are consumed by the softmax warps
+        // latent query chunks 0..7 -> TMEM columns [32c, 32c + 32) by tcgen05.cp;
+        // the copies execute in order with the MMAs below (and after the previous
+        // piece's MMAs, which still read the old query)
+        for (int c = 0; c < 8; ++c) {
+          if (!mbar_wait(ring_full0 + 8u * st.idx, st.phase, abortf, P.err, kErrWaitBase + 9))
+            return false;
+          tc_fence_after();
+          const uint64_t qd = ring_desc0 + (uint64_t)(st.idx * (kChunkBytes >> 4));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) tmem_cp_128x256b(tmem + kTmemQ + 32u * c + 8u * k, qd + 2 * k);
+          tc_commit(ring_empty0 + 8u * st.idx);
+          st.next(kRing);
+        }
         bool first = true;
         for (int pa = p0; pa < p1; pa += 2) {
           const int npg = (pa + 1 < p1) ? 2 : 1;
           const uint32_t idesc = npg == 2 ? idesc128 : idesc64;
           const bool last_pair = pa + 2 >= p1;
           ok = mbar_wait(bar(kBarSFree + sb.idx), sb.phase ^ 1u, abortf, P.err, kErrWaitBase + 4);
-          if (ok && first) {
-            ok = mbar_wait(bar(kBarQFull), q_phase, abortf, P.err, kErrWaitBase + 5);
-            q_phase ^= 1u;
-          }
           if (!ok) return false;
           const uint32_t dS = tmem + kTmemS + 128u * sb.idx;
           // the pair's 9 chunk stages, issued fully unrolled with precomputed
@@ -428,8 +445,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
       const float c = P.scale_log2;
       float* xmax = reinterpret_cast<float*>(smem + OFF_XCH);  // [2 pair parities][2 groups][128]
       float* xl = xmax + 4 * kRows;                            // [2][128] exact row sums
-      float* xlr = xl + 2 * kRows;                             // [2][128] rounded row sums
-      Ring st, sb;
+      Ring sb;
       uint32_t kp = 0;    // running page index of this cluster (P slot = kp % 4)
       uint32_t npair = 0; // running pair index (exchange-buffer parity)
       bool ok = true;
@@ -442,36 +458,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
       for_each_piece(P, it, [&](int b, int p0, int p1, int ordinal) {
         const int L = max(P.seqlens[b], 0);
         const int limit = valid ? (P.causal ? L - P.s_q + qi : L - 1) : -1;
-        // latent query chunks -> TMEM columns [32c, 32c + 32): group 0 copies
-        // chunks 0-3, group 1 chunks 4-7
-        {
-          Ring q = st;
-          q.advance(kRing, 4u * (uint32_t)wg);
-          for (int cc = 4 * wg; cc < 4 * wg + 4; ++cc) {
-            ok = named_bar_and(bar_all, 256, mbar_wait(bar(kBarRingFull + q.idx), q.phase, abortf, P.err,
-                                                       kErrWaitBase + 9));
-            if (!ok) return false;
-            const uint8_t* row = smem + OFF_RING + q.idx * kChunkBytes + r * 128;
-            uint32_t v[32];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const uint4 x = *reinterpret_cast<const uint4*>(row + ((u ^ (r & 7)) << 4));
-              v[4 * u] = x.x; v[4 * u + 1] = x.y; v[4 * u + 2] = x.z; v[4 * u + 3] = x.w;
-            }
-            tmem_st32(tmem + lane_off + kTmemQ + 32u * cc, v);
-            named_bar_sync(bar_wg, 128);
-            if (r == 0) mbar_arrive(bar(kBarRingEmpty + q.idx));
-            q.next(kRing);
-          }
-        }
-        st.advance(kRing, 8u + 9u * (uint32_t)((p1 - p0 + 1) / 2));  // page chunks: MMA thread's
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(kBarQFull));
-
-        // this group's share of the row sums: l exact (for lse), lr of the
-        // bf16-rounded weights the MMA multiplies (normalises O)
-        float m_ref = -INFINITY, l = 0.f, lr = 0.f;
+        // this group's share of the exact row sum l (for lse; the O-CTA sums the
+        // bf16-rounded weights that normalise O itself)
+        float m_ref = -INFINITY, l = 0.f;
         for (int pa = p0; pa < p1; pa += 2, ++npair) {
           const int npg = (pa + 1 < p1) ? 2 : 1;
           const bool last_pair = pa + 2 >= p1;
@@ -524,7 +513,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
               alpha = ex2(m_ref - mxs);
               resc = true;
               l *= alpha;
-              lr *= alpha;
             }
             m_ref = mxs;
           }
@@ -544,7 +532,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
           uint32_t pk[32];
           if (mine) {
             // P = exp2(S*c - base) -> bf16; masked entries are -inf and weigh exactly 0
-            float ls[4] = {0.f, 0.f, 0.f, 0.f}, lrs[4] = {0.f, 0.f, 0.f, 0.f};
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               float e0 = ex2(fmaf(__uint_as_float(s0[2 * j]), c, -base));
@@ -560,19 +548,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
               pk[j] = pack_bf16x2(e0, e1);
               pk[16 + j] = pack_bf16x2(e2, e3);
               ls[j & 3] += (e0 + e1) + (e2 + e3);
-              lrs[j & 3] += (__uint_as_float(pk[j] << 16) + __uint_as_float(pk[j] & 0xffff0000u)) +
-                            (__uint_as_float(pk[16 + j] << 16) + __uint_as_float(pk[16 + j] & 0xffff0000u));
             }
             l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-            lr += (lrs[0] + lrs[1]) + (lrs[2] + lrs[3]);
-          }
-          float ltot = 0.f, lrtot = 0.f;
-          if (last_pair) {  // the piece's totals: both groups' shares
-            xl[wg * kRows + r] = l;
-            xlr[wg * kRows + r] = lr;
-            named_bar_sync(bar_all, 256);
-            ltot = l + xl[(wg ^ 1) * kRows + r];
-            lrtot = lr + xlr[(wg ^ 1) * kRows + r];
           }
           if (mine) {
             // P row and the row's factors into the local staging buffers, then
@@ -584,7 +561,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
                   make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
             SideSlot* ss = reinterpret_cast<SideSlot*>(smem + OFF_STAGE_SIDE + buf * kSideBytes);
             ss->alpha[r] = wg == 0 ? alpha : 1.f;
-            ss->linv[r] = lrtot > 0.f ? 1.f / lrtot : 0.f;
             if (lane == 0) ss->wflag[warp & 3] = wg == 0 ? wany : 0u;
             fence_proxy_async_cta();  // staged data is read by the bulk copies (async proxy)
             named_bar_sync(bar_wg, 128);
@@ -596,7 +572,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
             }
           }
           kp += (uint32_t)npg;
+          if (last_pair) {  // the piece's row sum: both groups' shares
+            xl[wg * kRows + r] = l;
+            named_bar_sync(bar_all, 256);
+          }
           if (last_pair && valid && wg == 0) {
+            const float ltot = l + xl[kRows + r];
             const float lse_v = ltot > 0.f ? (m_ref + __log2f(ltot)) * kLn2 : -INFINITY;
             const int pslot = piece_slot(P, b, ordinal);
             if (pslot < 0)
@@ -626,9 +607,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
             const uint32_t fb = bar(kBarVFull + st.idx);
             mbar_arrive_expect_tx(fb, kVStageBytes);
             const uint32_t dst = sbase + OFF_V + st.idx * kVStageBytes;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              tma_load_3d(dst + j * kPageChunkBytes, &tmap_kv, fb, (4 * hh + j) * 64, g, page * kPage, pol);
+            // one box: 4 column chunks x 64 tokens, chunk-major in shared memory
+            tma_load_4d(dst, &tmap_v, fb, 0, page * kPage, 4 * hh, g, pol);
             issued[st.idx] = true;
             issued_phase[st.idx] = st.phase;
             st.next(kVStages);
@@ -660,12 +640,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
             done_phase ^= 1u;
             pending_epilogue = false;
             if (!ok) return false;
-          }
-          if (last) {  // keep this piece's 1/l: the side slot is recycled soon after
-            const float4* srcl = reinterpret_cast<const float4*>(side[ps].linv);
-            float4* dstl = reinterpret_cast<float4*>(mail->linv);
-#pragma unroll 4
-            for (int u = 0; u < kRows / 4; ++u) dstl[u] = srcl[u];
           }
           if (resc && !first) {
             // a row's reference max moved: finish all issued MMAs, rescale O rows
@@ -759,17 +733,47 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
       const bool valid = rr < P.R;
       const int qi = valid ? rr / P.hpk : 0;
       const int head = valid ? g * P.hpk + rr % P.hpk : 0;
-      uint32_t cmd_phase = 0;
-      for_each_piece(P, it, [&](int, int, int, int) {
-        for (;;) {
-          if (!__all_sync(0xffffffffu,
-                          mbar_wait(bar(kBarCmdFull), cmd_phase, abortf, P.err, kErrWaitBase + 20)))
+      uint32_t cmd_phase = 0, kp = 0, npiece = 0;
+      // P row r of each page, the 32 tokens of this group: 4 swizzled 16-byte chunks
+      const uint32_t prow_off = (uint32_t)((r >> 3) * 1024 + (r & 7) * 128);
+      // Both groups meet at named barrier 4 (256 threads), so every bounded wait
+      // is followed by an AND over all of them: all leave together or none.
+      auto agree = [&](bool ok) { return named_bar_and(4, 256, ok); };
+      // one command from the MMA thread
+      auto wait_cmd = [&]() {
+        if (!agree(mbar_wait(bar(kBarCmdFull), cmd_phase, abortf, P.err, kErrWaitBase + 20)))
+          return false;
+        cmd_phase ^= 1u;
+        tc_fence_after();
+        return true;
+      };
+      for_each_piece(P, it, [&](int, int p0, int p1, int) {
+        // lr: this group's half of the row's sum of the bf16 weights the MMA
+        // multiplies, rescaled with O
+        float lr = 0.f;
+        for (int p = p0; p < p1; ++p, ++kp) {
+          const uint32_t ps = kp % kPSlots, pph = (kp / kPSlots) & 1u;
+          if (!agree(mbar_wait<true>(bar(kBarPFull + ps), pph, abortf, P.err, kErrWaitBase + 23)))
             return false;
-          cmd_phase ^= 1u;
-          tc_fence_after();
-          const int cmd = *reinterpret_cast<volatile int*>(&mail->cmd);
-          if (cmd == kCmdRescale) {
-            const float a = side[mail->slot].alpha[r];
+          const volatile uint32_t* wf = side[ps].wflag;
+          const bool resc = p != p0 && (wf[0] | wf[1] | wf[2] | wf[3]) != 0u;
+          const float a = side[ps].alpha[r];
+          const uint8_t* prow = smem + OFF_P + ps * kPBytes + prow_off;
+          float s4[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 x = *reinterpret_cast<const uint4*>(prow + (((4 * wg + q) ^ (r & 7)) << 4));
+            s4[q] = ((__uint_as_float(x.x << 16) + __uint_as_float(x.x & 0xffff0000u)) +
+                     (__uint_as_float(x.y << 16) + __uint_as_float(x.y & 0xffff0000u))) +
+                    ((__uint_as_float(x.z << 16) + __uint_as_float(x.z & 0xffff0000u)) +
+                     (__uint_as_float(x.w << 16) + __uint_as_float(x.w & 0xffff0000u)));
+          }
+          lr = fmaf(lr, a, (s4[0] + s4[1]) + (s4[2] + s4[3]));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kBarPCons + ps));  // this warp is done with the slot
+          if (resc) {
+            // the MMA thread drains and posts a rescale before this page's MMAs
+            if (!wait_cmd()) return false;
             if (__any_sync(0xffffffffu, a != 1.f)) {  // tcgen05.ld/st are warp-collective
 #pragma unroll 1
               for (int j = 0; j < 8; ++j) {
@@ -783,46 +787,63 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
             }
             tc_fence_before();
             mbar_arrive(bar(kBarCmdDone));
-            continue;
           }
+        }
+        {
+          const bool okc = mbar_wait(bar(kBarCmdFull), cmd_phase, abortf, P.err, kErrWaitBase + 20);
+          float* xr = mail->lr_x[npiece & 1u][0];
+          xr[wg * kRows + r] = lr;  // exchanged with the other group at the barrier
+          if (!agree(okc)) return false;  // the piece's epilogue command
+          cmd_phase ^= 1u;
+          tc_fence_after();
+          const float lrt = lr + xr[(wg ^ 1) * kRows + r];
+          ++npiece;
           // epilogue: tcgen05.ld is warp-collective, so every thread loads and
           // only valid rows store
-          const float linv = mail->linv[r];
+          const float linv = lrt > 0.f ? 1.f / lrt : 0.f;
           const int b = mail->b;
           const int pslot = mail->part_slot;
+          // 64 accumulator columns per TMEM round trip
           if (pslot < 0) {
             uint16_t* dst = P.o + ((size_t)(b * P.s_q + qi) * P.h_q + head) * kDV + 256 * wg;
 #pragma unroll 1
-            for (int j = 0; j < 8; ++j) {
-              uint32_t v[32];
-              tmem_ld32_sync(tcol + 32 * j, v);
-              uint32_t pk[16];
+            for (int j = 0; j < 4; ++j) {
+              uint32_t v0[32], v1[32];
+              tmem_ld64_sync(tcol + 64 * j, v0, v1);
+              uint32_t pk[32];
 #pragma unroll
-              for (int u = 0; u < 16; ++u)
-                pk[u] = pack_bf16x2(__uint_as_float(v[2 * u]) * linv, __uint_as_float(v[2 * u + 1]) * linv);
+              for (int u = 0; u < 16; ++u) {
+                pk[u] = pack_bf16x2(__uint_as_float(v0[2 * u]) * linv, __uint_as_float(v0[2 * u + 1]) * linv);
+                pk[16 + u] =
+                    pack_bf16x2(__uint_as_float(v1[2 * u]) * linv, __uint_as_float(v1[2 * u + 1]) * linv);
+              }
               if (valid) {
-                st_global_v8(dst + 32 * j, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
-                st_global_v8(dst + 32 * j + 16, pk[8], pk[9], pk[10], pk[11], pk[12], pk[13], pk[14], pk[15]);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                  st_global_v8(dst + 64 * j + 16 * u, pk[8 * u], pk[8 * u + 1], pk[8 * u + 2], pk[8 * u + 3],
+                               pk[8 * u + 4], pk[8 * u + 5], pk[8 * u + 6], pk[8 * u + 7]);
               }
             }
           } else {
             float* dst = P.part_o + (((size_t)pslot * P.h_kv + g) * P.R + rr) * kDV + 256 * wg;
 #pragma unroll 1
-            for (int j = 0; j < 8; ++j) {
-              uint32_t v[32];
-              tmem_ld32_sync(tcol + 32 * j, v);
+            for (int j = 0; j < 4; ++j) {
+              uint32_t v[2][32];
+              tmem_ld64_sync(tcol + 64 * j, v[0], v[1]);
               if (valid) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                  st_global_v8(dst + 32 * j + 8 * u,
-                               __float_as_uint(__uint_as_float(v[8 * u]) * linv),
-                               __float_as_uint(__uint_as_float(v[8 * u + 1]) * linv),
-                               __float_as_uint(__uint_as_float(v[8 * u + 2]) * linv),
-                               __float_as_uint(__uint_as_float(v[8 * u + 3]) * linv),
-                               __float_as_uint(__uint_as_float(v[8 * u + 4]) * linv),
-                               __float_as_uint(__uint_as_float(v[8 * u + 5]) * linv),
-                               __float_as_uint(__uint_as_float(v[8 * u + 6]) * linv),
-                               __float_as_uint(__uint_as_float(v[8 * u + 7]) * linv));
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                  for (int u = 0; u < 4; ++u)
+                    st_global_v8(dst + 64 * j + 32 * h + 8 * u,
+                                 __float_as_uint(__uint_as_float(v[h][8 * u]) * linv),
+                                 __float_as_uint(__uint_as_float(v[h][8 * u + 1]) * linv),
+                                 __float_as_uint(__uint_as_float(v[h][8 * u + 2]) * linv),
+                                 __float_as_uint(__uint_as_float(v[h][8 * u + 3]) * linv),
+                                 __float_as_uint(__uint_as_float(v[h][8 * u + 4]) * linv),
+                                 __float_as_uint(__uint_as_float(v[h][8 * u + 5]) * linv),
+                                 __float_as_uint(__uint_as_float(v[h][8 * u + 6]) * linv),
+                                 __float_as_uint(__uint_as_float(v[h][8 * u + 7]) * linv));
               }
             }
           }
@@ -881,9 +902,9 @@ int decode_max_active_clusters(int device, int* out) {
 }
 
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, const CUtensorMap& tmap_q,
-                          cudaStream_t stream) {
+                          const CUtensorMap& tmap_v, cudaStream_t stream) {
   const int clusters = p.num_parts * p.h_kv * p.n_rg;
-  decode_kernel<<<2 * clusters, kThreads, SMEM_BYTES, stream>>>(tmap_kv, tmap_q, p);
+  decode_kernel<<<2 * clusters, kThreads, SMEM_BYTES, stream>>>(tmap_kv, tmap_q, tmap_v, p);
   return cudaGetLastError();
 }
 

@@ -13,6 +13,7 @@ constexpr int kD = 576;         // q/k width
 constexpr int kDV = 512;        // value width
 constexpr int kRows = 128;      // query rows per tile (the MMA's M)
 constexpr int kMetaInts = 8;    // int32 per scheduler part
+constexpr int kMaxParts = 2048; // scheduler parts one metadata kernel handles
 
 // Fixed cost, in pages, that the scheduler charges every piece of a sequence:
 // loading the 128x576 query tile (144 KB, two pages' worth of bytes), the
@@ -62,7 +63,7 @@ cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, in
 cudaError_t decode_prepare(int device);  // one-time per-device kernel attributes
 int decode_max_active_clusters(int device, int* out);
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, const CUtensorMap& tmap_q,
-                          cudaStream_t stream);
+                          const CUtensorMap& tmap_v, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 size_t decode_smem_bytes();
 

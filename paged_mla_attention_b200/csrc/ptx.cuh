@@ -120,21 +120,50 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with an explicit suspend-time hint: the thread sleeps in hardware
+// until the phase completes or `hint_ns` passes, instead of spinning.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster_sleep(uint32_t bar, uint32_t parity,
+                                                            uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Slow path of mbar_wait (kept out of line: it runs only when a phase has not
 // completed yet, and inlining it at every wait site bloats the hot loops).
+// Each try sleeps up to kWaitSliceNs in hardware, so a waiting warp takes
+// almost no issue slots from the warps that compute.
+constexpr uint32_t kWaitSliceNs = 20000;
 template <bool kClusterScope>
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                             int* err, int code) {
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > PMLA_WAIT_TIMEOUT_NS) {
-        *abort_flag = 1;
-        if (err) atomicCAS(err, 0, code);
-        return false;
-      }
+  for (;;) {
+    if (kClusterScope ? mbar_try_wait_cluster_sleep(bar, parity, kWaitSliceNs)
+                      : mbar_try_wait_sleep(bar, parity, kWaitSliceNs))
+      return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > PMLA_WAIT_TIMEOUT_NS) {
+      *abort_flag = 1;
+      if (err) atomicCAS(err, 0, code);
+      return false;
     }
   }
 }
@@ -215,6 +244,23 @@ __device__ __forceinline__ void tc_fence_after() {
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
+// 4-D tiled load into this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, uint32_t bar, int c0,
+                                            int c1, int c2, int c3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
+      : "memory");
+}
+
+// Asynchronous copy of a 128-row x 32-byte shared-memory tile (described by a
+// matrix descriptor, swizzle included) into TMEM: row i -> lane i, 8 columns.
+// Ordered with the tcgen05.mma instructions the same thread issues later.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // 3-D tiled load into this CTA's shared memory, completing `bytes` of

@@ -4,104 +4,204 @@
 // get_mla_metadata(cache_seqlens, s_q*h_q//h_kv, h_kv) returns
 // tile_scheduler_metadata and num_splits) and describe it as tiling /
 // load-balanced scheduling for variable-length sequences.  The algorithm here
-// is our own plain reading:
+// is our own plain reading, computed in parallel by one thread block:
 //
-//   cost(piece) = pages in the piece + kPieceCostPages
-//   target(p)   = ceil((remaining cost + expected split overhead) / parts
-//                 left), recomputed as each part starts, so rounding slack is
-//                 spread instead of piling up on the last part
+//   cost of a piece    = its pages + F               (F = kPieceCostPages)
+//   cost coordinate    = sequences laid end to end, each as F + its pages;
+//                        position (b, page) sits at X = S_b + F + page, the
+//                        start of sequence b at X = S_b
+//   total              = S_batch
+//   boundary of part p = X_p = floor(p (total + (P-1) F) / P) - (p-1) F
 //
-// Walk the sequences in order and fill part after part up to its target; a
-// sequence that does not fit in the rest of a part is cut, and the next part
-// continues it (one more piece, one more fixed cost).  Pieces shorter than two
-// pages are not cut off a sequence's tail.  The last part takes whatever is
-// left.  One thread does the walk: it is O(batch + parts) and runs once per
-// decode step, shared by all layers.
+// Every part is assumed to start inside a sequence and so pay one F of its
+// own; the spacing of the X_p gives each part the same share of the total plus
+// those P-1 overheads.  X_p is mapped back to (b, page) and snapped so that no
+// piece is shorter than two pages: a start at page 1 moves to the sequence
+// start, a start that would leave a one-page tail moves to the next sequence.
+// Snapping is monotone, so parts stay ordered (some may be empty).  When the
+// whole batch costs less than P (F + 1) the overhead assumption is dropped and
+// X_p = floor(p total / P).
+//
+// A part's cost is at most ceil((total + (P-1) F) / P) + F + 2 in either
+// regime; each thread finds its boundary by binary search, so the kernel
+// takes a few microseconds for any batch.
 #include "pagedmla_internal.cuh"
 
 namespace pmla {
 
-constexpr int kSchedThreads = 256;
-constexpr int kSchedSmemLens = 8192;  // lengths staged in shared memory (32 KB)
+constexpr int kSchedThreads = 1024;
+constexpr int kSchedWarps = kSchedThreads / 32;
+
+namespace {
+
+__device__ __forceinline__ int pages_of(const int32_t* seqlens, int b) {
+  const int L = seqlens[b] > 0 ? seqlens[b] : 0;
+  return (L + kPage - 1) / kPage;
+}
+
+// Exclusive block scan of one 64-bit value per thread (kSchedThreads threads).
+__device__ long long block_exclusive_scan(long long v, long long* warp_tot, long long* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long inc = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, inc, off);
+    if (lane >= off) inc += y;
+  }
+  if (lane == 31) warp_tot[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    long long t = warp_tot[lane];
+    long long ti = t;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, ti, off);
+      if (lane >= off) ti += y;
+    }
+    warp_tot[lane] = ti - t;  // exclusive prefix of the warp totals
+    if (lane == 31) *total = ti;
+  }
+  __syncthreads();
+  const long long r = warp_tot[warp] + inc - v;
+  __syncthreads();  // warp_tot may be reused by the caller's next scan
+  return r;
+}
+
+}  // namespace
 
 __global__ void __launch_bounds__(kSchedThreads) metadata_kernel(const int32_t* __restrict__ seqlens,
                                                                  int batch, int num_parts,
                                                                  int32_t* __restrict__ meta,
                                                                  int32_t* __restrict__ num_splits) {
-  // All threads stage the page counts in shared memory (coalesced loads) and
-  // reduce the total; thread 0 then walks them without global-memory latency.
-  __shared__ int32_t pages_s[kSchedSmemLens];
-  __shared__ long long partial[kSchedThreads / 32];
-  const long long fixed = kPieceCostPages;
-  const bool staged = batch <= kSchedSmemLens;
-  long long mine = 0;
-  for (int b = threadIdx.x; b < batch; b += kSchedThreads) {
-    const int L = seqlens[b] > 0 ? seqlens[b] : 0;
-    const int n = (L + kPage - 1) / kPage;
-    if (staged) pages_s[b] = n;
-    if (n > 0) mine += n + fixed;
+  __shared__ long long chunk_base[kSchedThreads];  // cost coordinate of each chunk's first sequence
+  __shared__ int chunk_ne[kSchedThreads];          // non-empty sequences before each chunk
+  __shared__ long long warp_tot[kSchedWarps];
+  __shared__ long long sh_total, sh_scratch;
+  __shared__ int start_b[kMaxParts + 1], start_pg[kMaxParts + 1];
+  __shared__ int cut_rank[kMaxParts + 1];  // cuts among parts <= p (inclusive)
+  __shared__ int cut_seq[kMaxParts];       // sequence of each distinct cut, in order
+  __shared__ int sh_ncuts;
+
+  const long long F = kPieceCostPages;
+  const int t = threadIdx.x;
+  const int P = num_parts;
+
+  // 1. every thread owns a contiguous chunk of sequences: chunk cost and
+  //    non-empty count, then block scans give each chunk's base
+  const int per = (batch + kSchedThreads - 1) / kSchedThreads;
+  const int c0 = min(t * per, batch), c1 = min(c0 + per, batch);
+  long long csum = 0;
+  int cne = 0;
+  for (int b = c0; b < c1; ++b) {
+    const int n = pages_of(seqlens, b);
+    if (n > 0) {
+      csum += n + F;
+      ++cne;
+    }
   }
-  for (int off = 16; off; off >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, off);
-  if ((threadIdx.x & 31) == 0) partial[threadIdx.x >> 5] = mine;
+  chunk_base[t] = block_exclusive_scan(csum, warp_tot, &sh_total);
+  chunk_ne[t] = (int)block_exclusive_scan(cne, warp_tot, &sh_scratch);
+  const long long total = sh_total;  // the scans end with a barrier
+
+  // 2. part boundaries
+  const long long A = total + (long long)(P - 1) * F;
+  const bool overhead_model = A >= (long long)P * (F + 1);
+  for (int p = t; p <= P; p += kSchedThreads) {
+    int sb = batch, spg = 0;
+    if (p == 0) {
+      sb = 0;
+    } else if (p < P) {
+      const long long X = overhead_model ? (long long)p * A / P - (long long)(p - 1) * F
+                                         : (long long)p * total / P;
+      if (X < total) {
+        // last chunk whose base is <= X (its cost is > 0 because X < total)
+        int lo = 0, hi = kSchedThreads - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (chunk_base[mid] <= X) lo = mid; else hi = mid - 1;
+        }
+        long long S = chunk_base[lo];
+        int b = min(lo * per, batch);
+        // the sequence containing X (empty sequences cost nothing and are skipped)
+        for (; b < batch; ++b) {
+          const int n = pages_of(seqlens, b);
+          const long long c = n > 0 ? n + F : 0;
+          if (X < S + c) {
+            long long pg = X - S - F;
+            if (pg < 2) pg = 0;
+            if (pg > 0 && n - pg < 2) {
+              sb = b + 1;
+              spg = 0;
+            } else {
+              sb = b;
+              spg = (int)pg;
+            }
+            break;
+          }
+          S += c;
+        }
+      }
+    }
+    start_b[p] = sb;
+    start_pg[p] = spg;
+  }
   __syncthreads();
-  if (threadIdx.x != 0) return;
-  auto pages_of = [&](int b) -> int {
-    if (staged) return pages_s[b];
-    const int L = seqlens[b] > 0 ? seqlens[b] : 0;
-    return (L + kPage - 1) / kPage;
-  };
-  // remaining cost: unassigned pages plus one fixed cost per sequence (or
-  // sequence remainder) that still has unassigned pages
-  long long remaining = 0;
-  for (int w = 0; w < kSchedThreads / 32; ++w) remaining += partial[w];
-  auto target_for = [&](int part) {
-    const long long left = num_parts - part;
-    long long t = (remaining + fixed * (left - 1) + left - 1) / left;
-    return t < fixed + 2 ? fixed + 2 : t;
+
+  // 3. distinct cut points (starts inside a sequence), ranked in order
+  if (t == 0) sh_ncuts = 0;
+  {
+    // parts are few (<= kMaxParts): each thread ranks a contiguous run of them
+    const int pp = (P + 1 + kSchedThreads - 1) / kSchedThreads;
+    const int q0 = min(t * pp, P + 1), q1 = min(q0 + pp, P + 1);
+    int mine = 0;
+    for (int p = q0; p < q1; ++p)
+      mine += (p > 0 && p < P && start_pg[p] > 0 &&
+               (start_b[p] != start_b[p - 1] || start_pg[p] != start_pg[p - 1]));
+    const long long before = block_exclusive_scan(mine, warp_tot, &sh_scratch);
+    int r = (int)before;
+    for (int p = q0; p < q1; ++p) {
+      const bool cut = p > 0 && p < P && start_pg[p] > 0 &&
+                       (start_b[p] != start_b[p - 1] || start_pg[p] != start_pg[p - 1]);
+      if (cut) cut_seq[r++] = start_b[p];
+      cut_rank[p] = r;
+    }
+    if (t == kSchedThreads - 1) sh_ncuts = r;
+  }
+  __syncthreads();
+  const int ncuts = sh_ncuts;
+  // number of cuts in sequences < b (lower bound) or <= b (upper bound)
+  auto cuts_before = [&](int b, bool inclusive) {
+    int lo = 0, hi = ncuts;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (inclusive ? cut_seq[mid] <= b : cut_seq[mid] < b) lo = mid + 1; else hi = mid;
+    }
+    return lo;
   };
 
-  int part = 0;
-  long long load = 0;
-  long long target = target_for(0);
-  int32_t* m = meta;
-  m[0] = 0; m[1] = 0; m[4] = 0; m[5] = 0; m[6] = 0; m[7] = 0;
-  num_splits[0] = 0;
-  int prefix = 0;  // running num_splits value (never re-read from global memory)
-  for (int b = 0; b < batch; ++b) {
-    const int n = pages_of(b);
-    int pieces = 0;
-    int p = 0;
-    while (p < n) {
-      const long long avail = target - load - fixed;
-      if (avail < 1 && load > 0 && part < num_parts - 1) {
-        // close this part at (b, p); the next one starts there
-        m[2] = b; m[3] = p;
-        remaining -= load;
-        if (p > 0) remaining += fixed;  // the rest of b becomes a new piece
-        ++part;
-        m = meta + (size_t)part * kMetaInts;
-        m[0] = b; m[1] = p; m[4] = pieces; m[5] = 0; m[6] = 0; m[7] = 0;
-        load = 0;
-        target = target_for(part);
-        continue;
-      }
-      int take = n - p;
-      if (part < num_parts - 1 && avail < take) {
-        take = (int)(avail < 1 ? 1 : avail);
-        if (n - p - take < 2) take = n - p;  // no tiny tail piece
-      }
-      p += take;
-      load += take + fixed;
-      ++pieces;
-    }
-    prefix += pieces;
-    num_splits[b + 1] = prefix;
+  // 4. metadata rows
+  for (int p = t; p < P; p += kSchedThreads) {
+    int32_t* m = meta + (size_t)p * kMetaInts;
+    const int b0 = start_b[p], pg0 = start_pg[p];
+    m[0] = b0;
+    m[1] = pg0;
+    m[2] = start_b[p + 1];
+    m[3] = start_pg[p + 1];
+    m[4] = pg0 > 0 ? cut_rank[p] - cuts_before(b0, false) : 0;
+    m[5] = 0;
+    m[6] = 0;
+    m[7] = 0;
   }
-  m[2] = batch; m[3] = 0;
-  for (int q = part + 1; q < num_parts; ++q) {
-    int32_t* e = meta + (size_t)q * kMetaInts;
-    e[0] = batch; e[1] = 0; e[2] = batch; e[3] = 0;
-    e[4] = 0; e[5] = 0; e[6] = 0; e[7] = 0;
+
+  // 5. num_splits = exclusive prefix of pieces: one per non-empty sequence plus
+  //    one per cut inside it
+  if (t == 0) num_splits[0] = 0;
+  int ne = chunk_ne[t];
+  int nc = c0 < c1 ? cuts_before(c0, false) : 0;
+  for (int b = c0; b < c1; ++b) {
+    ne += pages_of(seqlens, b) > 0;
+    while (nc < ncuts && cut_seq[nc] <= b) ++nc;
+    num_splits[b + 1] = ne + nc;
   }
 }
 

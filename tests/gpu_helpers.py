@@ -75,7 +75,7 @@ def check_schedule(meta, splits, seqlens, num_parts):
     """Invariants of the scheduler output (no numeric oracle exists for it):
     every page of every sequence is covered by exactly one part, in order;
     num_splits is the exclusive prefix sum of pieces; piece ordinals match;
-    and the heaviest part is within one piece's worth of the average."""
+    and no part costs more than the scheduler's stated bound."""
     seqlens = np.asarray(seqlens, dtype=np.int64)
     n = (np.maximum(seqlens, 0) + 63) // 64
     batch = len(n)
@@ -105,8 +105,10 @@ def check_schedule(meta, splits, seqlens, num_parts):
     for b in range(batch):
         assert np.all(covered[b] == 1), f"sequence {b}: pages not covered exactly once"
     assert np.array_equal(np.diff(splits), pieces), "num_splits is not the prefix sum of pieces"
-    # balance: no part is heavier than the mean part plus one piece's slack
-    avg = sum(loads) / num_parts
-    bound = max(avg * 1.1, 3 + 2) + 3 + 2
-    assert max(loads) <= bound, f"unbalanced parts: max {max(loads)} > {bound:.1f} (mean {avg:.1f})"
+    # balance: the scheduler's guarantee -- no part costs more than an even
+    # share of the total plus one overhead per possible cut, plus one piece's
+    # overhead and two pages of snapping
+    total = int(sum(int(x) + 3 for x in n if x > 0))
+    bound = -(-(total + (num_parts - 1) * 3) // num_parts) + 3 + 2
+    assert max(loads) <= bound, f"unbalanced parts: max {max(loads)} > {bound} (mean {sum(loads) / num_parts:.1f})"
     return loads
