@@ -11,10 +11,10 @@ needed between steps; the merge partials and q are small and may stay in L2.
 
 Prints ONE JSON line on rank 0.  ``value`` is the whole-job KV-read bandwidth
 (GB/s): KV bytes of all ranks' steps / max-over-ranks device time of the K
-timed steps.  Each step is replayed from a CUDA graph holding the three kernel
-launches.  ``roofline`` reports the decode call (split-KV kernel + merge
-kernel), timed per launch with CUDA events inside the timed region, against
-the measured HBM or bf16 peak.  ``e2e`` times the same step through the public
+timed steps.  Each step replays three CUDA graphs (schedule, decode kernel,
+merge kernel).  ``roofline`` reports the split-KV decode kernel, timed per
+launch with CUDA events inside the timed region, against the measured HBM or
+bf16 peak; ``us_per_call`` is decode + merge.  ``e2e`` times the same step through the public
 Python API from pinned host buffers (inputs copied in, o and lse copied out
 every step).  ``cpu_baseline`` times the fp64 oracle on the host cores on a
 bounded sample of the same workload.
@@ -89,6 +89,62 @@ def workload_desc(w: W.Workload) -> str:
             f"page=64 causal={w.causal} lengths={w.seqlen_kind}{list(w.seqlen_args)} bf16 N(0,1)")
 
 
+# ----------------------------------------------------------------------------- traffic
+KERNEL_SOURCES = ["decode.cu", "ptx.cuh", "pagedmla_internal.cuh"]
+
+
+def kernel_sources_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "paged_mla_attention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(config: str):
+    """DRAM bytes per decode-kernel launch from the committed ncu summary of this
+    workload, or None when there is none or the kernel sources changed since."""
+    path = os.path.join(ROOT, "profiles", f"decode_{config}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            parts = line.strip().split(":")
+            if len(parts) == 2 and parts[0] in ("traffic_bytes_per_launch", "kernel_sources_sha256_16"):
+                vals[parts[0]] = parts[1].strip()
+    if vals.get("kernel_sources_sha256_16") != kernel_sources_hash():
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ----------------------------------------------------------------------------- ranks
+def rank_inputs(w: W.Workload, rank: int) -> dict:
+    """Each rank decodes its own batch of the same workload (weak scaling): the
+    seed is offset by the rank, shapes and length distribution are shared."""
+    return W.make_inputs(w, seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank time over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, kv_bytes_per_rank: int, per_step_s: float) -> float:
+    """Whole-job KV-read bandwidth: every rank's KV bytes over the slowest rank's step time."""
+    return world * kv_bytes_per_rank / per_step_s / 1e9
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock and throttle reasons with NVML while the timed region runs."""
@@ -150,7 +206,7 @@ def bench_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = W.WORKLOADS[args.config]
-    inp = W.make_inputs(w, seed=w.seed + 1000 * rank)   # weak scaling: each rank its own batch
+    inp = rank_inputs(w, rank)   # weak scaling: each rank its own batch
     wc = work_counts(inp)
     peaks, peaks_src = load_peaks()
 
@@ -172,11 +228,11 @@ def bench_ours(args, rank, world, local_rank):
     def step_meta():
         meta_holder["m"], meta_holder["s"] = pm.get_mla_metadata(d["cache_seqlens"], R, inp["h_kv"])
 
-    def step_decode():
+    def step_decode(stage="all"):
         pm.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], W.D_V,
                                   meta_holder["m"], meta_holder["s"],
                                   softmax_scale=inp["softmax_scale"], causal=inp["causal"],
-                                  out=(o, lse), workspace=ws)
+                                  out=(o, lse), workspace=ws, stage=stage)
 
     if args.profile:
         # minimal plain-launch run for ncu: W warm-up steps then K steps, no graphs
@@ -202,21 +258,26 @@ def bench_ours(args, rank, world, local_rank):
     if err:
         raise RuntimeError(f"device error {err} during warm-up")
 
-    # capture the step as two CUDA graphs (schedule | decode + merge)
-    g_meta, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    # capture the step as three CUDA graphs (schedule | decode kernel | merge
+    # kernel) so that the decode kernel can be timed on its own
+    g_meta, g_dec, g_merge = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_meta, stream=stream):
         step_meta()
     with torch.cuda.graph(g_dec, stream=stream):
-        step_decode()
+        step_decode("decode")
+    with torch.cuda.graph(g_merge, stream=stream):
+        step_decode("merge")
     for _ in range(3):
         g_meta.replay()
         g_dec.replay()
+        g_merge.replay()
     torch.cuda.synchronize(dev)
 
     K = args.steps
     ev_start = torch.cuda.Event(enable_timing=True)
     ev_end = torch.cuda.Event(enable_timing=True)
     ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_m = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     if world > 1:
         import torch.distributed as dist
@@ -228,20 +289,20 @@ def bench_ours(args, rank, world, local_rank):
             g_meta.replay()
             ev_a[k].record()
             g_dec.replay()
+            ev_m[k].record()
+            g_merge.replay()
             ev_b[k].record()
         ev_end.record()
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     elapsed_ms = ev_start.elapsed_time(ev_end)
-    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]))
+    dec_ms = float(np.mean([a.elapsed_time(m) for a, m in zip(ev_a, ev_m)]))   # decode kernel
+    call_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]))  # decode + merge
     err = pm.device_error()
     if err:
         raise RuntimeError(f"device error {err} in the timed region")
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
 
     # end-to-end through the public API from pinned host buffers
     e2e_steps = max(3, min(K, args.e2e_steps))
@@ -270,10 +331,7 @@ def bench_ours(args, rank, world, local_rank):
     e1.record()
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev)
 
     # correctness spot-check of this very run against the oracle (rank 0, two sequences)
     spot = None
@@ -288,7 +346,7 @@ def bench_ours(args, rank, world, local_rank):
         spot = compare(og, lg, ro, rl, what="bench spot check")
 
     per_step_s = elapsed_ms / 1e3 / K
-    value = world * wc["kv_bytes"] / per_step_s / 1e9
+    value = whole_job_gbs(world, wc["kv_bytes"], per_step_s)
     dec_s = dec_ms / 1e3
     t_roof, bound = roofline_time(wc, peaks)
     if bound == "hbm":
@@ -305,12 +363,15 @@ def bench_ours(args, rank, world, local_rank):
                    "kv_tokens_per_gpu": wc["tokens"], "parallelism": f"replicas x{world} (batch-sharded, no exchange)",
                    "l2": "inputs (302 MB KV) larger than the 126 MB L2; no flush",
                    "step": "schedule + split-KV decode + merge, replayed from CUDA graphs"},
-        "us_per_call": round(dec_ms * 1e3, 3),
+        "us_decode_kernel": round(dec_ms * 1e3, 3),
+        "us_per_call": round(call_ms * 1e3, 3),
         "tflops": round(wc["flops"] / dec_s / 1e12, 2),
-        "kv_read_gbs_per_call": round(wc["kv_bytes"] / dec_s / 1e9, 1),
+        "kv_read_gbs_per_call": round(wc["kv_bytes"] / (call_ms / 1e3) / 1e9, 1),
         "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
-                     "frac": round(achieved / peak, 4), "traffic": args.traffic,
-                     "kernel": "decode call: split-KV decode kernel + merge kernel",
+                     "frac": round(achieved / peak, 4), "traffic": (args.traffic if args.traffic is not None
+                                                               else measured_traffic(args.config)),
+                     "traffic_unit": "bytes per launch (ncu dram read + write)",
+                     "kernel": "split-KV decode kernel (timed alone; the merge kernel follows it)",
                      "peak_source": f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback",
                      "roofline_us": round(t_roof * 1e6, 2),
                      "frac_of_roofline_time": round(t_roof / dec_s, 4)},

@@ -140,6 +140,35 @@ PMLA_API int mla_decode_with_kvcache(const uint16_t* q, const uint16_t* kvcache,
                             void* stream);
 
 /*
+ * The two kernels of mla_decode_with_kvcache as separate calls, with the same
+ * arguments, rules and errors; calling mla_decode_splits then mla_merge_splits
+ * on one stream equals one mla_decode_with_kvcache (the FlashMLA overview's
+ * split-KV kernel followed by its combine step, section 4.2(1)).
+ *
+ *   mla_decode_splits: the split-KV decode kernel only.  Sequences cut into
+ *       one piece get their final o and lse; pieces of split sequences leave
+ *       normalised fp32 partials and their lse in `workspace`.
+ *   mla_merge_splits: the merge kernel only.  Reads those partials from
+ *       `workspace` and writes o and lse of split and of empty sequences.
+ * Useful to time the decode kernel on its own; no state is kept between the
+ * calls other than the caller's workspace, which must not change in between.
+ */
+PMLA_API int mla_decode_splits(const uint16_t* q, const uint16_t* kvcache, const int32_t* block_table,
+                               const int32_t* cache_seqlens, int batch, int s_q, int h_q, int h_kv,
+                               int d, int dv, int num_pages, int max_pages_per_seq,
+                               const int32_t* tile_scheduler_metadata, int num_parts,
+                               const int32_t* num_splits, int causal, float softmax_scale,
+                               uint16_t* o, float* lse, void* workspace, size_t workspace_bytes,
+                               void* stream);
+PMLA_API int mla_merge_splits(const uint16_t* q, const uint16_t* kvcache, const int32_t* block_table,
+                              const int32_t* cache_seqlens, int batch, int s_q, int h_q, int h_kv,
+                              int d, int dv, int num_pages, int max_pages_per_seq,
+                              const int32_t* tile_scheduler_metadata, int num_parts,
+                              const int32_t* num_splits, int causal, float softmax_scale,
+                              uint16_t* o, float* lse, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
  * Allocation-free variant of mla_decode_with_kvcache (the FlashMLA pages have
  * no counterpart: this entry point exists for callers that cannot allocate
  * device memory, such as code inside a CUDA stream capture, runtimes that own

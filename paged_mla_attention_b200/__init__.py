@@ -55,9 +55,10 @@ def _load() -> ctypes.CDLL:
     lib.mla_get_metadata_sizes.restype = I
     lib.mla_get_metadata.argtypes = [P, I, I, I, P, I, P, P]
     lib.mla_get_metadata.restype = I
-    lib.mla_decode_with_kvcache.argtypes = [P, P, P, P] + [I] * 8 + [P, I, P, I, ctypes.c_float,
-                                                                     P, P, P, SZ, P]
-    lib.mla_decode_with_kvcache.restype = I
+    for name in ("mla_decode_with_kvcache", "mla_decode_splits", "mla_merge_splits"):
+        fn = getattr(lib, name)
+        fn.argtypes = [P, P, P, P] + [I] * 8 + [P, I, P, I, ctypes.c_float, P, P, P, SZ, P]
+        fn.restype = I
     lib.pmla_device_error.argtypes = []
     lib.pmla_device_error.restype = I
     lib.pmla_last_error.argtypes = []
@@ -67,7 +68,20 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
-library = _load()
+class _Library:
+    """The C library, loaded on first use (so that the build module, which lives
+    in this package, can run before the library exists).  Any use raises
+    ImportError when the library is missing: there is no fallback path."""
+
+    _lib = None
+
+    def __getattr__(self, name):
+        if _Library._lib is None:
+            _Library._lib = _load()
+        return getattr(_Library._lib, name)
+
+
+library = _Library()
 
 
 def _check(rc: int) -> None:
@@ -129,7 +143,7 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
                            tile_scheduler_metadata: torch.Tensor, num_splits: torch.Tensor,
                            softmax_scale: Optional[float] = None, causal: bool = False,
                            out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
-                           workspace: Optional[torch.Tensor] = None
+                           workspace: Optional[torch.Tensor] = None, stage: str = "all"
                            ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Paged MLA decode.
 
@@ -140,8 +154,15 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
     head_dim_v  512
     Returns o bf16 [batch, s_q, h_q, 512] and lse fp32 [batch, h_q, s_q] (natural log).
     softmax_scale defaults to 1/sqrt(192).  ``out`` and ``workspace`` may be
-    passed to avoid per-call allocation.
+    passed to avoid per-call allocation.  ``stage`` selects the C entry point:
+    "all" (mla_decode_with_kvcache), "decode" (mla_decode_splits, the decode
+    kernel alone) or "merge" (mla_merge_splits, the merge kernel alone; pass the
+    same ``out`` and ``workspace`` as the "decode" call).
     """
+    fn = {"all": library.mla_decode_with_kvcache, "decode": library.mla_decode_splits,
+          "merge": library.mla_merge_splits}.get(stage)
+    if fn is None:
+        raise ValueError(f"stage must be 'all', 'decode' or 'merge', got {stage!r}")
     _need(q, "q", torch.bfloat16, 4)
     _need(kvcache, "kvcache", torch.bfloat16, 4)
     _need(block_table, "block_table", torch.int32, 2)
@@ -172,7 +193,7 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
             o, lse = out
         if workspace is None or workspace.numel() < ws_bytes:
             workspace = torch.empty((max(ws_bytes, 16),), dtype=torch.uint8, device=dev)
-        _check(library.mla_decode_with_kvcache(
+        _check(fn(
             _ptr(q), _ptr(kvcache), _ptr(block_table), _ptr(cache_seqlens), batch, s_q, h_q, h_kv,
             d, head_dim_v, num_pages, block_table.shape[1], _ptr(tile_scheduler_metadata), num_parts,
             _ptr(num_splits), int(bool(causal)), scale, _ptr(o), _ptr(lse), _ptr(workspace),

@@ -163,13 +163,19 @@ int mla_get_metadata(const int32_t* cache_seqlens, int batch, int num_heads_per_
   return PMLA_OK;
 }
 
-int mla_decode_with_kvcache(const uint16_t* q, const uint16_t* kvcache, const int32_t* block_table,
-                            const int32_t* cache_seqlens, int batch, int s_q, int h_q, int h_kv,
-                            int d, int dv, int num_pages, int max_pages_per_seq,
-                            const int32_t* tile_scheduler_metadata, int num_parts,
-                            const int32_t* num_splits, int causal, float softmax_scale,
-                            uint16_t* o, float* lse, void* workspace, size_t workspace_bytes,
-                            void* stream) {
+}  // extern "C"
+
+namespace {
+
+constexpr int kStageDecode = 1, kStageMerge = 2;
+
+// Shared body of the three decode entry points: validates everything, then
+// launches the split-KV decode kernel and/or the merge kernel.
+int decode_impl(const uint16_t* q, const uint16_t* kvcache, const int32_t* block_table,
+                const int32_t* cache_seqlens, int batch, int s_q, int h_q, int h_kv, int d, int dv,
+                int num_pages, int max_pages_per_seq, const int32_t* tile_scheduler_metadata,
+                int num_parts, const int32_t* num_splits, int causal, float softmax_scale, uint16_t* o,
+                float* lse, void* workspace, size_t workspace_bytes, void* stream, int stages) {
   g_last_error.clear();
   if (d != PMLA_HEAD_DIM || dv != PMLA_HEAD_DIM_V)
     return fail(PMLA_ERR_UNSUPPORTED, "head dims must be d=576, dv=512 (got %d, %d)", d, dv);
@@ -210,105 +216,131 @@ int mla_decode_with_kvcache(const uint16_t* q, const uint16_t* kvcache, const in
   DeviceInfo* info;
   int rc = device_setup(&dev, &info);
   if (rc) return rc;
-  auto encode = get_encode();
-  if (!encode) return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-
-  // kvcache as a 3-D tensor: [576 columns] x [h_kv heads] x [num_pages*64 tokens];
-  // each TMA box is 64 columns x 1 head x 64 tokens with the 128-byte swizzle.
-  CUtensorMap tmap;
-  cuuint64_t gdim[3] = {(cuuint64_t)pmla::kD, (cuuint64_t)h_kv,
-                        (cuuint64_t)num_pages * pmla::kPage};
-  cuuint64_t gstride[2] = {(cuuint64_t)pmla::kD * 2, (cuuint64_t)h_kv * pmla::kD * 2};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)pmla::kPage};
-  cuuint32_t estride[3] = {1, 1, 1};
-  CUresult cr = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(kvcache),
-                       gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)cr);
-
-  // kvcache once more as a 4-D tensor [64 columns] x [tokens] x [9 column chunks]
-  // x [h_kv heads] (the chunk stride, 128 bytes, is below the token stride): one
-  // box of 64 columns x 64 tokens x 4 chunks lands as 4 chunk-major 8 KB tiles,
-  // i.e. half of a page's value part in a single TMA instruction.
-  CUtensorMap tmap_v;
-  {
-    cuuint64_t vdim[4] = {64, (cuuint64_t)num_pages * pmla::kPage, (cuuint64_t)pmla::kD / 64,
-                          (cuuint64_t)h_kv};
-    cuuint64_t vstride[3] = {(cuuint64_t)h_kv * pmla::kD * 2, 128, (cuuint64_t)pmla::kD * 2};
-    cuuint32_t vbox[4] = {64, (cuuint32_t)pmla::kPage, 4, 1};
-    cuuint32_t vestride[4] = {1, 1, 1, 1};
-    cr = encode(&tmap_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t*>(kvcache), vdim,
-                vstride, vbox, vestride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (cr != CUDA_SUCCESS)
-      return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled (value tiles) failed (%d)", (int)cr);
-  }
-
-  // q as a 2-D tensor: [576 columns] x [batch*s_q*h_q rows]; boxes of 64 columns
-  // x min(h_q/h_kv, 128) rows with the 128-byte swizzle.
-  CUtensorMap tmap_q;
-  {
-    const int hpk = h_q / h_kv;
-    cuuint64_t qdim[2] = {(cuuint64_t)pmla::kD, (cuuint64_t)batch * s_q * h_q};
-    cuuint64_t qstride[1] = {(cuuint64_t)pmla::kD * 2};
-    cuuint32_t qbox[2] = {64, (cuuint32_t)(hpk < pmla::kRows ? hpk : pmla::kRows)};
-    cuuint32_t qestride[2] = {1, 1};
-    cr = encode(&tmap_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(q), qdim,
-                qstride, qbox, qestride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (cr != CUDA_SUCCESS)
-      return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled (q) failed (%d)", (int)cr);
-  }
-
-  pmla::DecodeParams p;
-  p.q = q;
-  p.block_table = block_table;
-  p.seqlens = cache_seqlens;
-  p.meta = tile_scheduler_metadata;
-  p.num_splits = num_splits;
-  p.o = o;
-  p.lse = lse;
-  p.part_o = static_cast<float*>(workspace);
-  p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + lse_off);
-  p.err = info->err_ptr;
-  p.batch = batch;
-  p.s_q = s_q;
-  p.h_q = h_q;
-  p.h_kv = h_kv;
-  p.hpk = h_q / h_kv;
-  p.R = (int)R;
-  p.n_rg = (int)((R + pmla::kRows - 1) / pmla::kRows);
-  p.num_parts = num_parts;
-  p.max_pages = max_pages_per_seq;
-  p.num_pages = num_pages;
-  p.causal = causal ? 1 : 0;
-  p.scale_log2 = softmax_scale * 1.4426950408889634f;
-  if ((long long)num_parts * h_kv * p.n_rg > (1ll << 30))
-    return fail(PMLA_ERR_UNSUPPORTED, "grid too large");
-
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = pmla::decode_prepare(dev);
-  if (e != cudaSuccess) return fail_cuda(e, "decode kernel attributes");
-  e = pmla::launch_decode(p, tmap, tmap_q, tmap_v, st);
-  if (e != cudaSuccess) return fail_cuda(e, "decode kernel launch");
+  if (stages & kStageDecode) {
+    auto encode = get_encode();
+    if (!encode) return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
 
+    // kvcache as a 3-D tensor: [576 columns] x [h_kv heads] x [num_pages*64 tokens];
+    // each TMA box is 64 columns x 1 head x 64 tokens with the 128-byte swizzle.
+    CUtensorMap tmap;
+    cuuint64_t gdim[3] = {(cuuint64_t)pmla::kD, (cuuint64_t)h_kv,
+                          (cuuint64_t)num_pages * pmla::kPage};
+    cuuint64_t gstride[2] = {(cuuint64_t)pmla::kD * 2, (cuuint64_t)h_kv * pmla::kD * 2};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)pmla::kPage};
+    cuuint32_t estride[3] = {1, 1, 1};
+    CUresult cr = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(kvcache),
+                         gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)cr);
+
+    // kvcache once more as a 4-D tensor [64 columns] x [tokens] x [9 column chunks]
+    // x [h_kv heads] (the chunk stride, 128 bytes, is below the token stride): one
+    // box of 64 columns x 64 tokens x 4 chunks lands as 4 chunk-major 8 KB tiles,
+    // i.e. half of a page's value part in a single TMA instruction.
+    CUtensorMap tmap_v;
+    {
+      cuuint64_t vdim[4] = {64, (cuuint64_t)num_pages * pmla::kPage, (cuuint64_t)pmla::kD / 64,
+                            (cuuint64_t)h_kv};
+      cuuint64_t vstride[3] = {(cuuint64_t)h_kv * pmla::kD * 2, 128, (cuuint64_t)pmla::kD * 2};
+      cuuint32_t vbox[4] = {64, (cuuint32_t)pmla::kPage, 4, 1};
+      cuuint32_t vestride[4] = {1, 1, 1, 1};
+      cr = encode(&tmap_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t*>(kvcache), vdim,
+                  vstride, vbox, vestride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (cr != CUDA_SUCCESS)
+        return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled (value tiles) failed (%d)", (int)cr);
+  }
+
+    // q as a 2-D tensor: [576 columns] x [batch*s_q*h_q rows]; boxes of 64 columns
+    // x min(h_q/h_kv, 128) rows with the 128-byte swizzle.
+    CUtensorMap tmap_q;
+    {
+      const int hpk = h_q / h_kv;
+      cuuint64_t qdim[2] = {(cuuint64_t)pmla::kD, (cuuint64_t)batch * s_q * h_q};
+      cuuint64_t qstride[1] = {(cuuint64_t)pmla::kD * 2};
+      cuuint32_t qbox[2] = {64, (cuuint32_t)(hpk < pmla::kRows ? hpk : pmla::kRows)};
+      cuuint32_t qestride[2] = {1, 1};
+      cr = encode(&tmap_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(q), qdim,
+                  qstride, qbox, qestride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (cr != CUDA_SUCCESS)
+        return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled (q) failed (%d)", (int)cr);
+  }
+
+    pmla::DecodeParams p;
+    p.q = q;
+    p.block_table = block_table;
+    p.seqlens = cache_seqlens;
+    p.meta = tile_scheduler_metadata;
+    p.num_splits = num_splits;
+    p.o = o;
+    p.lse = lse;
+    p.part_o = static_cast<float*>(workspace);
+    p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + lse_off);
+    p.err = info->err_ptr;
+    p.batch = batch;
+    p.s_q = s_q;
+    p.h_q = h_q;
+    p.h_kv = h_kv;
+    p.hpk = h_q / h_kv;
+    p.R = (int)R;
+    p.n_rg = (int)((R + pmla::kRows - 1) / pmla::kRows);
+    p.num_parts = num_parts;
+    p.max_pages = max_pages_per_seq;
+    p.num_pages = num_pages;
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    if ((long long)num_parts * h_kv * p.n_rg > (1ll << 30))
+      return fail(PMLA_ERR_UNSUPPORTED, "grid too large");
+
+    cudaError_t e = pmla::decode_prepare(dev);
+    if (e != cudaSuccess) return fail_cuda(e, "decode kernel attributes");
+    e = pmla::launch_decode(p, tmap, tmap_q, tmap_v, st);
+    if (e != cudaSuccess) return fail_cuda(e, "decode kernel launch");
+  }
+  if (!(stages & kStageMerge)) return PMLA_OK;
+
+  size_t lse_off2;
+  workspace_for(batch, (int)R, h_kv, num_parts, &lse_off2);
   pmla::CombineParams c;
   c.num_splits = num_splits;
-  c.part_o = p.part_o;
-  c.part_lse = p.part_lse;
+  c.part_o = static_cast<float*>(workspace);
+  c.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + lse_off2);
   c.o = o;
   c.lse = lse;
   c.batch = batch;
   c.s_q = s_q;
   c.h_q = h_q;
   c.h_kv = h_kv;
-  c.hpk = p.hpk;
-  c.R = p.R;
-  e = pmla::launch_combine(c, st);
+  c.hpk = h_q / h_kv;
+  c.R = (int)R;
+  cudaError_t e = pmla::launch_combine(c, st);
   if (e != cudaSuccess) return fail_cuda(e, "combine kernel launch");
   return PMLA_OK;
 }
+
+}  // namespace
+
+extern "C" {
+
+#define PMLA_DECODE_ARGS                                                                       \
+  q, kvcache, block_table, cache_seqlens, batch, s_q, h_q, h_kv, d, dv, num_pages,              \
+      max_pages_per_seq, tile_scheduler_metadata, num_parts, num_splits, causal, softmax_scale, \
+      o, lse, workspace, workspace_bytes, stream
+#define PMLA_DECODE_PARAMS                                                                     \
+  const uint16_t *q, const uint16_t *kvcache, const int32_t *block_table,                      \
+      const int32_t *cache_seqlens, int batch, int s_q, int h_q, int h_kv, int d, int dv,      \
+      int num_pages, int max_pages_per_seq, const int32_t *tile_scheduler_metadata,            \
+      int num_parts, const int32_t *num_splits, int causal, float softmax_scale, uint16_t *o,  \
+      float *lse, void *workspace, size_t workspace_bytes, void *stream
+
+int mla_decode_with_kvcache(PMLA_DECODE_PARAMS) {
+  return decode_impl(PMLA_DECODE_ARGS, kStageDecode | kStageMerge);
+}
+int mla_decode_splits(PMLA_DECODE_PARAMS) { return decode_impl(PMLA_DECODE_ARGS, kStageDecode); }
+int mla_merge_splits(PMLA_DECODE_PARAMS) { return decode_impl(PMLA_DECODE_ARGS, kStageMerge); }
 
 int pmla_device_error(void) {
   int dev;

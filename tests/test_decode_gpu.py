@@ -52,6 +52,29 @@ def test_non_causal_multi_token():
     _check(_small([5, 90, 300], s_q=2, h_q=64, causal=False, seed=21), "s_q=2 non-causal")
 
 
+def test_two_stage_calls_equal_the_single_call():
+    # mla_decode_splits then mla_merge_splits == mla_decode_with_kvcache, bit for bit
+    import torch
+    import paged_mla_attention_b200 as pm
+    inp = _small([9000, 100, 3000, 0, 64, 1], h_q=128, seed=23)
+    d = to_device(inp)
+    meta, splits = pm.get_mla_metadata(d["cache_seqlens"], 128, 1)
+    assert int((splits[1:] - splits[:-1]).max()) >= 2
+    args = (d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], W.D_V, meta, splits)
+    o1, l1 = pm.flash_mla_with_kvcache(*args, softmax_scale=inp["softmax_scale"])
+    ws = torch.empty((pm.workspace_bytes(inp["batch"], 1, 128, 1),), dtype=torch.uint8, device="cuda")
+    o2 = torch.full_like(o1, float("nan"))
+    l2 = torch.full_like(l1, float("nan"))
+    pm.flash_mla_with_kvcache(*args, softmax_scale=inp["softmax_scale"], out=(o2, l2), workspace=ws,
+                              stage="decode")
+    pm.flash_mla_with_kvcache(*args, softmax_scale=inp["softmax_scale"], out=(o2, l2), workspace=ws,
+                              stage="merge")
+    torch.cuda.synchronize()
+    assert pm.device_error() == 0
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(l1.view(torch.int32), l2.view(torch.int32))
+
+
 def test_split_sequences_merge():
     # long sequences next to short ones: pieces of the long ones go through the merge kernel
     stats, meta, splits = _check(_small([9000, 100, 3000, 64, 1], h_q=128, seed=22), "splits")
