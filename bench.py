@@ -11,10 +11,11 @@ needed between steps; the merge partials and q are small and may stay in L2.
 
 Prints ONE JSON line on rank 0.  ``value`` is the whole-job KV-read bandwidth
 (GB/s): KV bytes of all ranks' steps / max-over-ranks device time of the K
-timed steps.  Each step replays three CUDA graphs (schedule, decode kernel,
-merge kernel).  ``roofline`` reports the split-KV decode kernel, timed per
-launch with CUDA events inside the timed region, against the measured HBM or
-bf16 peak; ``us_per_call`` is decode + merge.  ``e2e`` times the same step through the public
+timed steps.  Each step replays two CUDA graphs: the schedule, and the decode
+call (decode kernel, then the merge kernel launched as its programmatic
+dependent).  ``roofline`` reports the split-KV decode kernel, replayed alone K
+times right after the timed steps with CUDA events around each launch, against
+the measured HBM or bf16 peak; ``us_per_call`` is the decode call.  ``e2e`` times the same step through the public
 Python API from pinned host buffers (inputs copied in, o and lse copied out
 every step).  ``cpu_baseline`` times the fp64 oracle on the host cores on a
 bounded sample of the same workload.
@@ -258,26 +259,26 @@ def bench_ours(args, rank, world, local_rank):
     if err:
         raise RuntimeError(f"device error {err} during warm-up")
 
-    # capture the step as three CUDA graphs (schedule | decode kernel | merge
-    # kernel) so that the decode kernel can be timed on its own
-    g_meta, g_dec, g_merge = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    # CUDA graphs: the schedule; the decode call (decode kernel, then the merge
+    # kernel as a programmatic dependent that overlaps the decode tail); and the
+    # decode kernel alone, for the roofline
+    g_meta, g_all, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_meta, stream=stream):
         step_meta()
+    with torch.cuda.graph(g_all, stream=stream):
+        step_decode("all")
     with torch.cuda.graph(g_dec, stream=stream):
         step_decode("decode")
-    with torch.cuda.graph(g_merge, stream=stream):
-        step_decode("merge")
     for _ in range(3):
         g_meta.replay()
+        g_all.replay()
         g_dec.replay()
-        g_merge.replay()
     torch.cuda.synchronize(dev)
 
     K = args.steps
     ev_start = torch.cuda.Event(enable_timing=True)
     ev_end = torch.cuda.Event(enable_timing=True)
     ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_m = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     if world > 1:
         import torch.distributed as dist
@@ -288,17 +289,23 @@ def bench_ours(args, rank, world, local_rank):
         for k in range(K):
             g_meta.replay()
             ev_a[k].record()
-            g_dec.replay()
-            ev_m[k].record()
-            g_merge.replay()
+            g_all.replay()
             ev_b[k].record()
         ev_end.record()
+        torch.cuda.synchronize(dev)
+        # the decode kernel alone, K more launches right after the timed steps
+        # (same stream, same inputs), each bracketed by events
+        ev_c = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+        ev_c[0].record()
+        for k in range(K):
+            g_dec.replay()
+            ev_c[k + 1].record()
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     elapsed_ms = ev_start.elapsed_time(ev_end)
-    dec_ms = float(np.mean([a.elapsed_time(m) for a, m in zip(ev_a, ev_m)]))   # decode kernel
     call_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]))  # decode + merge
+    dec_ms = float(np.mean([ev_c[k].elapsed_time(ev_c[k + 1]) for k in range(K)]))  # decode kernel
     err = pm.device_error()
     if err:
         raise RuntimeError(f"device error {err} in the timed region")
@@ -378,7 +385,7 @@ def bench_ours(args, rank, world, local_rank):
         "e2e": {"value": round(world * wc["kv_bytes"] / (e2e_ms / 1e3 / e2e_steps) / 1e9, 3), "unit": "GB/s",
                 "steps": e2e_steps, "ms_per_step": round(e2e_ms / e2e_steps, 4),
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
-        "gpu_launches": 3 * K,
+        "gpu_launches": 3 * K,  # schedule, decode, merge per timed step
         "clocks": clk.summary(),
     }
     if spot is not None:

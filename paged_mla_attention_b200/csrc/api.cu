@@ -16,6 +16,22 @@
 #include "../../include/pagedmla.h"
 #include "pagedmla_internal.cuh"
 
+namespace pmla {
+
+WorkspaceLayout workspace_layout(int batch, int R, int h_kv, int num_parts) {
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  WorkspaceLayout w;
+  const size_t slots = (size_t)batch + (size_t)num_parts;
+  const size_t rows = slots * (size_t)h_kv * (size_t)R;
+  w.lse_off = rows * kDV * sizeof(float);
+  w.done_off = w.lse_off + up(rows * sizeof(float));
+  w.done_count = (size_t)batch * (size_t)h_kv * (size_t)((R + kRows - 1) / kRows);
+  w.bytes = w.done_off + up(w.done_count * sizeof(int));
+  return w;
+}
+
+}  // namespace pmla
+
 namespace {
 
 thread_local std::string g_last_error;
@@ -98,11 +114,9 @@ int parts_for(const DeviceInfo& d, int num_heads_per_head_k, int num_heads_k) {
 }
 
 size_t workspace_for(int batch, int R, int h_kv, int num_parts, size_t* lse_offset) {
-  const size_t slots = (size_t)batch + (size_t)num_parts;
-  const size_t rows = slots * (size_t)h_kv * (size_t)R;
-  const size_t o_bytes = rows * pmla::kDV * sizeof(float);
-  *lse_offset = o_bytes;
-  return o_bytes + ((rows * sizeof(float) + 255) & ~size_t(255));
+  const pmla::WorkspaceLayout w = pmla::workspace_layout(batch, R, h_kv, num_parts);
+  *lse_offset = w.lse_off;
+  return w.bytes;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -279,6 +293,8 @@ int decode_impl(const uint16_t* q, const uint16_t* kvcache, const int32_t* block
     p.lse = lse;
     p.part_o = static_cast<float*>(workspace);
     p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + lse_off);
+    const pmla::WorkspaceLayout wl = pmla::workspace_layout(batch, (int)R, h_kv, num_parts);
+    p.seq_done = reinterpret_cast<int*>(static_cast<char*>(workspace) + wl.done_off);
     p.err = info->err_ptr;
     p.batch = batch;
     p.s_q = s_q;
@@ -297,17 +313,21 @@ int decode_impl(const uint16_t* q, const uint16_t* kvcache, const int32_t* block
 
     cudaError_t e = pmla::decode_prepare(dev);
     if (e != cudaSuccess) return fail_cuda(e, "decode kernel attributes");
+    // the merge kernel counts completion signals from zero
+    e = cudaMemsetAsync(p.seq_done, 0, wl.done_count * sizeof(int), st);
+    if (e != cudaSuccess) return fail_cuda(e, "clearing the completion counters");
     e = pmla::launch_decode(p, tmap, tmap_q, tmap_v, st);
     if (e != cudaSuccess) return fail_cuda(e, "decode kernel launch");
   }
   if (!(stages & kStageMerge)) return PMLA_OK;
 
-  size_t lse_off2;
-  workspace_for(batch, (int)R, h_kv, num_parts, &lse_off2);
+  const pmla::WorkspaceLayout wl2 = pmla::workspace_layout(batch, (int)R, h_kv, num_parts);
   pmla::CombineParams c;
   c.num_splits = num_splits;
   c.part_o = static_cast<float*>(workspace);
-  c.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + lse_off2);
+  c.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + wl2.lse_off);
+  c.seq_done = reinterpret_cast<const int*>(static_cast<char*>(workspace) + wl2.done_off);
+  c.err = info->err_ptr;
   c.o = o;
   c.lse = lse;
   c.batch = batch;
@@ -316,6 +336,7 @@ int decode_impl(const uint16_t* q, const uint16_t* kvcache, const int32_t* block
   c.h_kv = h_kv;
   c.hpk = h_q / h_kv;
   c.R = (int)R;
+  c.n_rg = (int)((R + pmla::kRows - 1) / pmla::kRows);
   cudaError_t e = pmla::launch_combine(c, st);
   if (e != cudaSuccess) return fail_cuda(e, "combine kernel launch");
   return PMLA_OK;

@@ -9,10 +9,22 @@
 // Sequences with no pages at all (n = 0) also get o = 0, lse = -inf here;
 // unsplit sequences (n = 1) were written by the decode kernel directly.
 //
-// Layout: one warp per query row, each lane owns 16 of the 512 columns (four
-// float4 per partial), so every partial row is read with fully coalesced
-// 2 KB warp loads.  Grid: (row blocks of 8, h_kv, batch).
+// Layout: the partials are chunk-major, [slot][h_kv][64 chunks of 8 columns]
+// [R rows][8].  A block takes 32 consecutive rows of one (sequence, KV head);
+// warp w handles chunks w, w+8, ..., lane = row, so every load is 1 KB
+// contiguous.  The merged rows go through shared memory and leave as
+// contiguous 16-byte stores.  Grid: (row blocks of 32, h_kv, batch).
+//
+// Overlap with the decode kernel: this kernel is launched as a programmatic
+// dependent of the decode kernel, which lets it start once every decode CTA is
+// resident.  Each finished split piece adds 2 to a counter per (sequence, KV
+// head, row group) -- once after its lse, once after its o rows, each behind
+// a device-scope fence -- and a block merges only after the counter reaches
+// 2 x pieces (a bounded wait that records an error if it runs out).  Blocks
+// end by waiting for the whole decode grid, so work queued after this kernel
+// still sees the decode kernel complete.
 #include "pagedmla_internal.cuh"
+#include "ptx.cuh"
 
 #include <cuda_bf16.h>
 
@@ -20,76 +32,149 @@ namespace pmla {
 
 namespace {
 
-constexpr int kRowsPerBlock = 8;  // 8 warps, one row each
+constexpr int kMergeRows = 32;
+constexpr int kMergeThreads = 256;
+constexpr int kChunks = kDV / 8;  // 64 chunks of 8 columns
+constexpr int kMaxPieces = 64;    // lse values staged in shared memory per round
 
-__global__ void __launch_bounds__(32 * kRowsPerBlock)
-combine_kernel(const CombineParams P) {
+__global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombineParams P) {
+  // merged rows, bf16; rows padded by 16 bytes so the lane-per-row stores hit distinct banks
+  __shared__ __align__(16) uint16_t tile[kMergeRows][kDV + 8];
+  __shared__ float row_lse[kMergeRows];
   const int b = blockIdx.z;
   const int g = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rr = blockIdx.x * kRowsPerBlock + warp;
-  if (rr >= P.R) return;
+  const int r0 = blockIdx.x * kMergeRows;
   const int s0 = P.num_splits[b];
   const int n = P.num_splits[b + 1] - s0;
-  if (n == 1) return;
-  const int qi = rr / P.hpk;
-  const int head = g * P.hpk + rr % P.hpk;
-  uint4* orow = reinterpret_cast<uint4*>(P.o + ((size_t)(b * P.s_q + qi) * P.h_q + head) * kDV) +
-                lane * 2;
-  float* lse_out = P.lse + ((size_t)b * P.h_q + head) * P.s_q + qi;
-
-  float m = -INFINITY;
-  for (int k = lane; k < n; k += 32)
-    m = fmaxf(m, P.part_lse[((size_t)(s0 + k) * P.h_kv + g) * P.R + rr]);
-#pragma unroll
-  for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  if (n == 0 || m == -INFINITY) {
-    orow[0] = make_uint4(0, 0, 0, 0);
-    orow[1] = make_uint4(0, 0, 0, 0);
-    if (lane == 0) *lse_out = -INFINITY;
+  if (n == 1) {  // written by the decode kernel directly
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     return;
   }
-  float z = 0.f;
-  for (int k = lane; k < n; k += 32)
-    z += __expf(P.part_lse[((size_t)(s0 + k) * P.h_kv + g) * P.R + rr] - m);
-#pragma unroll
-  for (int off = 16; off; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-  const float total = m + __logf(z);
+  const int rr = r0 + lane;
+  const bool valid = rr < P.R;
+  __shared__ int ready;
+  if (n >= 2) {
+    if (threadIdx.x == 0) {
+      const int* ctr = P.seq_done + ((size_t)b * P.h_kv + g) * P.n_rg + r0 / kRows;
+      const uint64_t t0 = global_timer_ns();
+      int ok = 1;
+      for (;;) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+        if (v >= 2 * n) break;
+        if (global_timer_ns() - t0 > PMLA_WAIT_TIMEOUT_NS) {
+          atomicCAS(P.err, 0, kErrWaitBase + 30);
+          ok = 0;
+          break;
+        }
+        __nanosleep(256);
+      }
+      ready = ok;
+    }
+    __syncthreads();
+    if (!ready) return;
+  }
 
-  float acc[16];
-#pragma unroll
-  for (int u = 0; u < 16; ++u) acc[u] = 0.f;
-  for (int k = 0; k < n; ++k) {
-    const size_t row = ((size_t)(s0 + k) * P.h_kv + g) * P.R + rr;
-    const float w = __expf(P.part_lse[row] - total);
-    const float4* src = reinterpret_cast<const float4*>(P.part_o + row * kDV) + lane * 4;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float4 v = __ldg(src + u);
-      acc[4 * u] = fmaf(w, v.x, acc[4 * u]);
-      acc[4 * u + 1] = fmaf(w, v.y, acc[4 * u + 1]);
-      acc[4 * u + 2] = fmaf(w, v.z, acc[4 * u + 2]);
-      acc[4 * u + 3] = fmaf(w, v.w, acc[4 * u + 3]);
+  // all lse_k of the block's rows in one round trip (warp w loads pieces w, w+8,
+  // ...), then every thread derives its row's total and the merge weights from
+  // shared memory; pieces beyond kMaxPieces go round again
+  __shared__ float wsh[kMaxPieces][kMergeRows];
+  float m = -INFINITY, z = 0.f;
+  for (int k0 = 0; k0 < n; k0 += kMaxPieces) {
+    const int nk = min(n - k0, kMaxPieces);
+    __syncthreads();
+    for (int k = warp; k < nk; k += 8)
+      wsh[k][lane] = valid ? __ldcg(P.part_lse + ((size_t)(s0 + k0 + k) * P.h_kv + g) * P.R + rr)
+                           : -INFINITY;
+    __syncthreads();
+    for (int k = 0; k < nk; ++k) {  // online max / sum of exp over this row's pieces
+      const float x = wsh[k][lane];
+      if (x > m) {
+        z = z * __expf(m - x) + 1.f;
+        m = x;
+      } else if (x != -INFINITY) {
+        z += __expf(x - m);
+      }
     }
   }
-  uint32_t pk[8];
+  const float total = (m == -INFINITY) ? -INFINITY : m + __logf(z);
+  if (warp == 0) row_lse[lane] = total;
+
+  float acc[8][8];
 #pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * u], acc[2 * u + 1]);
-    pk[u] = *reinterpret_cast<uint32_t*>(&h2);
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc[i][u] = 0.f;
+  if (valid && total != -INFINITY) {
+    for (int k = 0; k < n; ++k) {
+      const size_t slot = (size_t)(s0 + k) * P.h_kv + g;
+      const float w = __expf((n <= kMaxPieces ? wsh[k][lane] : __ldcg(P.part_lse + slot * P.R + rr)) - total);
+      const float4* src = reinterpret_cast<const float4*>(P.part_o + (slot * kChunks * P.R + rr) * 8);
+      float4 x[8], y[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {  // all 16 loads in flight before any use
+        const float4* c = src + (size_t)(warp + 8 * i) * P.R * 2;
+        x[i] = __ldcg(c);  // written by a kernel still running: L2, not the L1 cache
+        y[i] = __ldcg(c + 1);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        acc[i][0] = fmaf(w, x[i].x, acc[i][0]);
+        acc[i][1] = fmaf(w, x[i].y, acc[i][1]);
+        acc[i][2] = fmaf(w, x[i].z, acc[i][2]);
+        acc[i][3] = fmaf(w, x[i].w, acc[i][3]);
+        acc[i][4] = fmaf(w, y[i].x, acc[i][4]);
+        acc[i][5] = fmaf(w, y[i].y, acc[i][5]);
+        acc[i][6] = fmaf(w, y[i].z, acc[i][6]);
+        acc[i][7] = fmaf(w, y[i].w, acc[i][7]);
+      }
+    }
   }
-  orow[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-  orow[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-  if (lane == 0) *lse_out = total;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint32_t pk[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[i][2 * u], acc[i][2 * u + 1]);
+      pk[u] = *reinterpret_cast<uint32_t*>(&h2);
+    }
+    *reinterpret_cast<uint4*>(&tile[lane][(warp + 8 * i) * 8]) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+  __syncthreads();
+
+  // rows r0.. of (b, g): row rr is query token rr / hpk, head g*hpk + rr % hpk
+  constexpr int kVec = kDV * 2 / 16;  // 16-byte pieces per row
+  for (int e = threadIdx.x; e < kMergeRows * kVec; e += kMergeThreads) {
+    const int row = e / kVec, c = e % kVec;
+    const int r = r0 + row;
+    if (r >= P.R) continue;
+    const int qi = r / P.hpk, head = g * P.hpk + r % P.hpk;
+    uint4* dst = reinterpret_cast<uint4*>(P.o + ((size_t)(b * P.s_q + qi) * P.h_q + head) * kDV) + c;
+    *dst = *reinterpret_cast<const uint4*>(&tile[row][c * 8]);
+  }
+  if (warp == 0 && valid) {
+    const int qi = rr / P.hpk, head = g * P.hpk + rr % P.hpk;
+    P.lse[((size_t)b * P.h_q + head) * P.s_q + qi] = row_lse[lane];
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace
 
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
-  dim3 grid((p.R + kRowsPerBlock - 1) / kRowsPerBlock, p.h_kv, p.batch);
   if (p.batch == 0) return cudaSuccess;
-  combine_kernel<<<grid, 32 * kRowsPerBlock, 0, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((p.R + kMergeRows - 1) / kMergeRows, p.h_kv, p.batch);
+  cfg.blockDim = dim3(kMergeThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, p);
 }
 
 }  // namespace pmla

@@ -275,6 +275,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
   cluster_wait();
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem_base;
+  // every CTA of this grid is resident now: the merge kernel, launched as a
+  // programmatic dependent, may start on SMs as they free up (it waits for the
+  // completion signals of the pieces it merges)
+  if (tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const PartIter it(P, part);
   const uint32_t peer = rank ^ 1u;
 
@@ -576,14 +580,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
             xl[wg * kRows + r] = l;
             named_bar_sync(bar_all, 256);
           }
-          if (last_pair && valid && wg == 0) {
-            const float ltot = l + xl[kRows + r];
-            const float lse_v = ltot > 0.f ? (m_ref + __log2f(ltot)) * kLn2 : -INFINITY;
+          if (last_pair && wg == 0) {
             const int pslot = piece_slot(P, b, ordinal);
-            if (pslot < 0)
-              P.lse[((size_t)b * P.h_q + head) * P.s_q + qi] = lse_v;
-            else
-              P.part_lse[((size_t)pslot * P.h_kv + g) * P.R + rr] = lse_v;
+            if (valid) {
+              const float ltot = l + xl[kRows + r];
+              const float lse_v = ltot > 0.f ? (m_ref + __log2f(ltot)) * kLn2 : -INFINITY;
+              if (pslot < 0)
+                P.lse[((size_t)b * P.h_q + head) * P.s_q + qi] = lse_v;
+              else
+                P.part_lse[((size_t)pslot * P.h_kv + g) * P.R + rr] = lse_v;
+            }
+            if (pslot >= 0) {  // split piece: signal the merge kernel (lse half)
+              __threadfence();
+              named_bar_sync(bar_wg, 128);
+              if (r == 0) atomicAdd(&P.seq_done[((size_t)b * P.h_kv + g) * P.n_rg + rg], 1);
+            }
           }
         }
         return true;
@@ -825,7 +836,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
               }
             }
           } else {
-            float* dst = P.part_o + (((size_t)pslot * P.h_kv + g) * P.R + rr) * kDV + 256 * wg;
+            // partials are chunk-major, [slot][h_kv][64 chunks of 8 columns][R][8], so
+            // the 32 rows of a warp store 1 KB contiguous per chunk
+            float* dst = P.part_o + (((size_t)pslot * P.h_kv + g) * (kDV / 8) + 32 * wg) * P.R * 8 +
+                         (size_t)rr * 8;
+            const size_t cstride = (size_t)P.R * 8;  // floats between consecutive chunks
 #pragma unroll 1
             for (int j = 0; j < 4; ++j) {
               uint32_t v[2][32];
@@ -835,7 +850,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
                 for (int h = 0; h < 2; ++h)
 #pragma unroll
                   for (int u = 0; u < 4; ++u)
-                    st_global_v8(dst + 64 * j + 32 * h + 8 * u,
+                    st_global_v8(dst + (8 * j + 4 * h + u) * cstride,
                                  __float_as_uint(__uint_as_float(v[h][8 * u]) * linv),
                                  __float_as_uint(__uint_as_float(v[h][8 * u + 1]) * linv),
                                  __float_as_uint(__uint_as_float(v[h][8 * u + 2]) * linv),
@@ -846,6 +861,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
                                  __float_as_uint(__uint_as_float(v[h][8 * u + 7]) * linv));
               }
             }
+            // signal the merge kernel (partial o half) once all 256 threads stored
+            __threadfence();
+            named_bar_sync(4, 256);
+            if (tid == 128) atomicAdd(&P.seq_done[((size_t)b * P.h_kv + g) * P.n_rg + rg], 1);
           }
           tc_fence_before();
           mbar_arrive(bar(kBarCmdDone));

@@ -53,8 +53,8 @@ PMLA_API int mla_decode_with_kvcache_noalloc(
   if (h_kv >= 1 && h_q >= 1 && h_q % h_kv == 0 && batch >= 0 && num_parts >= 1 && s_q >= 1) {
     // the same upper bound mla_get_metadata_sizes reports for this shape
     const size_t R = (size_t)s_q * (size_t)(h_q / h_kv);
-    const size_t rows = ((size_t)batch + (size_t)num_parts) * (size_t)h_kv * R;
-    const size_t need = rows * pmla::kDV * sizeof(float) + ((rows * sizeof(float) + 255) & ~size_t(255));
+    const size_t need = R > (size_t(1) << 20) ? ~size_t(0)
+                        : pmla::workspace_layout(batch, (int)R, h_kv, num_parts).bytes;
     if (need > kNoAllocScratchBytes) {
       char msg[256];
       snprintf(msg, sizeof msg,

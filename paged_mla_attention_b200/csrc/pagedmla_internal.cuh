@@ -39,6 +39,7 @@ struct DecodeParams {
   float* lse;                   // [b][h_q][s_q]
   float* part_o;                // [slots][h_kv][R][512]
   float* part_lse;              // [slots][h_kv][R]
+  int* seq_done;                // [b][h_kv][n_rg] completion signals of split pieces
   int* err;                     // device error word
   int batch, s_q, h_q, h_kv;
   int hpk;                      // h_q / h_kv
@@ -52,10 +53,20 @@ struct CombineParams {
   const int32_t* num_splits;
   const float* part_o;
   const float* part_lse;
+  const int* seq_done;          // [b][h_kv][n_rg]: 2 signals per finished split piece
+  int* err;                     // device error word
   uint16_t* o;
   float* lse;
-  int batch, s_q, h_q, h_kv, hpk, R;
+  int batch, s_q, h_q, h_kv, hpk, R, n_rg;
 };
+
+// Workspace layout of one decode call: split partials o (chunk-major fp32),
+// their lse, and the per-(sequence, KV head, row group) completion counters the
+// merge kernel waits on.  Returns the total size.
+struct WorkspaceLayout {
+  size_t lse_off, done_off, done_count, bytes;
+};
+WorkspaceLayout workspace_layout(int batch, int R, int h_kv, int num_parts);
 
 // Host launchers (each returns the CUDA error of its launch).
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* meta,
