@@ -337,6 +337,7 @@ int decode_impl(const uint16_t* q, const uint16_t* kvcache, const int32_t* block
   c.hpk = h_q / h_kv;
   c.R = (int)R;
   c.n_rg = (int)((R + pmla::kRows - 1) / pmla::kRows);
+  c.num_parts = num_parts;
   cudaError_t e = pmla::launch_combine(c, st);
   if (e != cudaSuccess) return fail_cuda(e, "combine kernel launch");
   return PMLA_OK;

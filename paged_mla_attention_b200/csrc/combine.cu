@@ -10,10 +10,12 @@
 // unsplit sequences (n = 1) were written by the decode kernel directly.
 //
 // Layout: the partials are chunk-major, [slot][h_kv][64 chunks of 8 columns]
-// [R rows][8].  A block takes 32 consecutive rows of one (sequence, KV head);
-// warp w handles chunks w, w+8, ..., lane = row, so every load is 1 KB
-// contiguous.  The merged rows go through shared memory and leave as
-// contiguous 16-byte stores.  Grid: (row blocks of 32, h_kv, batch).
+// [R rows][8].  A block takes 32 consecutive rows and one eighth (64) of the
+// columns of one (sequence, KV head); warp w handles chunk w of that slice,
+// lane = row, so every load is 1 KB contiguous, and 8 pieces' loads are in
+// flight at once.  The merged rows go through shared memory and leave as
+// contiguous 16-byte stores.  Grid: (row blocks of 32 x 8 column slices, h_kv,
+// batch).
 //
 // Overlap with the decode kernel: this kernel is launched as a programmatic
 // dependent of the decode kernel, which lets it start once every decode CTA is
@@ -35,16 +37,26 @@ namespace {
 constexpr int kMergeRows = 32;
 constexpr int kMergeThreads = 256;
 constexpr int kChunks = kDV / 8;  // 64 chunks of 8 columns
-constexpr int kMaxPieces = 64;    // lse values staged in shared memory per round
 
+// kQuarters column slices per row block (one block each; a warp handles
+// kCPW = 8 / kQuarters chunks of its slice) and kPieceBatch pieces whose loads
+// are in flight together.  Few slices suit sequences cut into few pieces (less
+// repeated lse work, fewer blocks waiting); many slices suit a long sequence
+// cut into many pieces, whose merge would otherwise run on a handful of SMs.
+template <int kQuarters, int kPieceBatch>
 __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombineParams P) {
+  constexpr int kQCols = kDV / kQuarters;
+  constexpr int kQChunks = kChunks / kQuarters;
+  constexpr int kCPW = kQChunks / 8;  // chunks per warp
+  constexpr int kMaxPieces = kQuarters == 1 ? 64 : 128;  // lse values staged per round
   // merged rows, bf16; rows padded by 16 bytes so the lane-per-row stores hit distinct banks
-  __shared__ __align__(16) uint16_t tile[kMergeRows][kDV + 8];
+  __shared__ __align__(16) uint16_t tile[kMergeRows][kQCols + 8];
   __shared__ float row_lse[kMergeRows];
   const int b = blockIdx.z;
   const int g = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r0 = blockIdx.x * kMergeRows;
+  const int r0 = (blockIdx.x / kQuarters) * kMergeRows;
+  const int quarter = blockIdx.x % kQuarters;
   const int s0 = P.num_splits[b];
   const int n = P.num_splits[b + 1] - s0;
   if (n == 1) {  // written by the decode kernel directly
@@ -101,38 +113,56 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombinePar
   const float total = (m == -INFINITY) ? -INFINITY : m + __logf(z);
   if (warp == 0) row_lse[lane] = total;
 
-  float acc[8][8];
+  float acc[kCPW][8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < kCPW; ++i)
 #pragma unroll
     for (int u = 0; u < 8; ++u) acc[i][u] = 0.f;
   if (valid && total != -INFINITY) {
-    for (int k = 0; k < n; ++k) {
-      const size_t slot = (size_t)(s0 + k) * P.h_kv + g;
-      const float w = __expf((n <= kMaxPieces ? wsh[k][lane] : __ldcg(P.part_lse + slot * P.R + rr)) - total);
-      const float4* src = reinterpret_cast<const float4*>(P.part_o + (slot * kChunks * P.R + rr) * 8);
-      float4 x[8], y[8];
+    // pieces go kPieceBatch at a time so that 16 loads per thread are in flight
+    const float4* base = reinterpret_cast<const float4*>(P.part_o) +
+                         ((size_t)(quarter * kQChunks + warp) * P.R + rr) * 2;
+    const size_t piece_stride = (size_t)P.h_kv * kChunks * P.R * 2;  // float4s between slots
+    const size_t chunk8 = (size_t)8 * P.R * 2;                       // float4s between chunks c, c+8
+    for (int k0 = 0; k0 < n; k0 += kPieceBatch) {
+      float w[kPieceBatch];
+      float4 x[kPieceBatch][kCPW], y[kPieceBatch][kCPW];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {  // all 16 loads in flight before any use
-        const float4* c = src + (size_t)(warp + 8 * i) * P.R * 2;
-        x[i] = __ldcg(c);  // written by a kernel still running: L2, not the L1 cache
-        y[i] = __ldcg(c + 1);
+      for (int j = 0; j < kPieceBatch; ++j) {
+        const int k = k0 + j;
+        w[j] = 0.f;
+        if (k < n) {
+          const size_t slot = (size_t)(s0 + k) * P.h_kv + g;
+          const float lk = n <= kMaxPieces ? wsh[k][lane] : __ldcg(P.part_lse + slot * P.R + rr);
+          w[j] = __expf(lk - total);
+          const float4* src = base + (size_t)(s0 + k) * piece_stride + (size_t)g * kChunks * P.R * 2;
+#pragma unroll
+          for (int i = 0; i < kCPW; ++i) {  // written by a kernel still running: L2, not the L1 cache
+            x[j][i] = __ldcg(src + i * chunk8);
+            y[j][i] = __ldcg(src + i * chunk8 + 1);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < kCPW; ++i) x[j][i] = y[j][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        acc[i][0] = fmaf(w, x[i].x, acc[i][0]);
-        acc[i][1] = fmaf(w, x[i].y, acc[i][1]);
-        acc[i][2] = fmaf(w, x[i].z, acc[i][2]);
-        acc[i][3] = fmaf(w, x[i].w, acc[i][3]);
-        acc[i][4] = fmaf(w, y[i].x, acc[i][4]);
-        acc[i][5] = fmaf(w, y[i].y, acc[i][5]);
-        acc[i][6] = fmaf(w, y[i].z, acc[i][6]);
-        acc[i][7] = fmaf(w, y[i].w, acc[i][7]);
-      }
+      for (int j = 0; j < kPieceBatch; ++j)
+#pragma unroll
+        for (int i = 0; i < kCPW; ++i) {
+          acc[i][0] = fmaf(w[j], x[j][i].x, acc[i][0]);
+          acc[i][1] = fmaf(w[j], x[j][i].y, acc[i][1]);
+          acc[i][2] = fmaf(w[j], x[j][i].z, acc[i][2]);
+          acc[i][3] = fmaf(w[j], x[j][i].w, acc[i][3]);
+          acc[i][4] = fmaf(w[j], y[j][i].x, acc[i][4]);
+          acc[i][5] = fmaf(w[j], y[j][i].y, acc[i][5]);
+          acc[i][6] = fmaf(w[j], y[j][i].z, acc[i][6]);
+          acc[i][7] = fmaf(w[j], y[j][i].w, acc[i][7]);
+        }
     }
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < kCPW; ++i) {
     uint32_t pk[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -144,16 +174,17 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombinePar
   __syncthreads();
 
   // rows r0.. of (b, g): row rr is query token rr / hpk, head g*hpk + rr % hpk
-  constexpr int kVec = kDV * 2 / 16;  // 16-byte pieces per row
+  constexpr int kVec = kQCols * 2 / 16;  // 16-byte pieces per row of the quarter
   for (int e = threadIdx.x; e < kMergeRows * kVec; e += kMergeThreads) {
     const int row = e / kVec, c = e % kVec;
     const int r = r0 + row;
     if (r >= P.R) continue;
     const int qi = r / P.hpk, head = g * P.hpk + r % P.hpk;
-    uint4* dst = reinterpret_cast<uint4*>(P.o + ((size_t)(b * P.s_q + qi) * P.h_q + head) * kDV) + c;
+    uint4* dst =
+        reinterpret_cast<uint4*>(P.o + ((size_t)(b * P.s_q + qi) * P.h_q + head) * kDV + quarter * kQCols) + c;
     *dst = *reinterpret_cast<const uint4*>(&tile[row][c * 8]);
   }
-  if (warp == 0 && valid) {
+  if (warp == 0 && valid && quarter == 0) {
     const int qi = rr / P.hpk, head = g * P.hpk + rr % P.hpk;
     P.lse[((size_t)b * P.h_q + head) * P.s_q + qi] = row_lse[lane];
   }
@@ -165,7 +196,11 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombinePar
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
   if (p.batch == 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((p.R + kMergeRows - 1) / kMergeRows, p.h_kv, p.batch);
+  // a long sequence cut into many pieces shows as many scheduler parts per
+  // sequence: spread each row block over 8 column slices then
+  const bool many = p.num_parts >= 2 * p.batch;
+  const int slices = many ? 8 : 1;
+  cfg.gridDim = dim3(((p.R + kMergeRows - 1) / kMergeRows) * slices, p.h_kv, p.batch);
   cfg.blockDim = dim3(kMergeThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
@@ -174,7 +209,8 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, combine_kernel, p);
+  return many ? cudaLaunchKernelEx(&cfg, combine_kernel<8, 8>, p)
+              : cudaLaunchKernelEx(&cfg, combine_kernel<1, 1>, p);
 }
 
 }  // namespace pmla

@@ -57,7 +57,7 @@ struct CombineParams {
   int* err;                     // device error word
   uint16_t* o;
   float* lse;
-  int batch, s_q, h_q, h_kv, hpk, R, n_rg;
+  int batch, s_q, h_q, h_kv, hpk, R, n_rg, num_parts;
 };
 
 // Workspace layout of one decode call: split partials o (chunk-major fp32),
