@@ -157,6 +157,30 @@ def test_scheduler_invariants(seed):
             check_schedule(meta.cpu().numpy(), splits.cpu().numpy(), lens, meta.shape[0])
 
 
+def test_scheduler_exhaustive_small():
+    """Every length vector with batch <= 4 over lengths {0, 1, 64, 65, 129, 256}, for
+    1, 2, 5 and 74 parts, through the C entry point: coverage, ordinals, prefix sums
+    and the stated balance bound all hold."""
+    import ctypes
+    import itertools
+    import torch
+    import paged_mla_attention_b200 as pm
+    vals = [0, 1, 64, 65, 129, 256]
+    lib = pm.library
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for batch in range(1, 5):
+        for lens in itertools.product(vals, repeat=batch):
+            sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+            for parts in (1, 2, 5, 74):
+                meta = torch.empty((parts, 8), dtype=torch.int32, device="cuda")
+                splits = torch.empty((batch + 1,), dtype=torch.int32, device="cuda")
+                rc = lib.mla_get_metadata(ctypes.c_void_p(sl.data_ptr()), batch, 128, 1,
+                                          ctypes.c_void_p(meta.data_ptr()), parts,
+                                          ctypes.c_void_p(splits.data_ptr()), stream)
+                assert rc == 0
+                check_schedule(meta.cpu().numpy(), splits.cpu().numpy(), np.array(lens), parts)
+
+
 FULL = ["uniform", "varlen", "causal2", "skew"]
 
 
