@@ -53,6 +53,8 @@ class OracleLib:
         lib.oracle_mla_combine.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = I
+        lib.oracle_append_kvcache.argtypes = [P, P, P] + [I] * 7 + [P]
+        lib.oracle_append_kvcache.restype = I
         self.lib = lib
         self.path = path
 
@@ -99,6 +101,24 @@ class OracleLib:
         self.lib.oracle_mla_combine(_ptr(part_o), _ptr(part_lse), n, dv, _ptr(o), _ptr(lse))
         return o, float(lse[0])
 
+    def append_kvcache(self, new_kv: np.ndarray, block_table: np.ndarray, cache_seqlens: np.ndarray,
+                       kvcache: np.ndarray) -> Tuple[np.ndarray, bool]:
+        """Reference append: returns (a new cache with the tokens written, all rows written?).
+
+        new_kv: uint16 bf16 bits [b][s_new][h_kv][d]; kvcache: uint16 [pages][page][h_kv][d]
+        (not modified); cache_seqlens: lengths before the append.
+        """
+        new_kv = np.ascontiguousarray(new_kv, dtype=np.uint16)
+        out = np.array(kvcache, dtype=np.uint16, copy=True, order="C")
+        block_table = np.ascontiguousarray(block_table, dtype=np.int32)
+        cache_seqlens = np.ascontiguousarray(cache_seqlens, dtype=np.int32)
+        b, s_new, h_kv, d = new_kv.shape
+        pages, page, h_kv2, d2 = out.shape
+        assert h_kv2 == h_kv and d2 == d and block_table.shape[0] == b
+        rc = self.lib.oracle_append_kvcache(_ptr(new_kv), _ptr(block_table), _ptr(cache_seqlens), b,
+                                            s_new, h_kv, d, page, block_table.shape[1], pages, _ptr(out))
+        return out, rc == 0
+
     def decode_inputs(self, inp: dict, nthreads: int = 0, **kw) -> Tuple[np.ndarray, np.ndarray]:
         """Run on an input dict from ``mla_workloads.make_inputs``."""
         return self.mla_decode(inp["q"], inp["kvcache"], inp["block_table"],
@@ -126,6 +146,10 @@ def mla_decode(*a, **kw):
 
 def mla_combine(*a, **kw):
     return default().mla_combine(*a, **kw)
+
+
+def append_kvcache(*a, **kw):
+    return default().append_kvcache(*a, **kw)
 
 
 def decode_inputs(inp: dict, nthreads: int = 0, **kw):

@@ -165,3 +165,43 @@ void oracle_mla_combine(const double* part_o, const double* part_lse, int n, int
   }
   *lse = total;
 }
+
+/*
+ * Appending new tokens to the paged cache (the write side of the same paged
+ * layout, FlashMLA overview section 4.2(1): logical 64-token blocks mapped to
+ * physical blocks by block_table).  Token t (0-based) of the s_new new tokens
+ * of sequence b sits at position L_b + t of that sequence, i.e. in physical
+ * page block_table[b][(L_b + t) / page_size], slot (L_b + t) % page_size, and
+ * its row [c^KV ; k^R] for KV head g is copied there unchanged.
+ *
+ * A row whose position lies beyond the block table (>= max_pages*page_size)
+ * or whose page id is outside [0, num_pages) is not written; the function then
+ * returns -1 (0 when every row was written).
+ */
+int oracle_append_kvcache(const uint16_t* new_kv, const int32_t* block_table,
+                          const int32_t* seqlens, int batch, int s_new, int h_kv, int d,
+                          int page_size, int max_pages, int num_pages, uint16_t* kvcache) {
+  int bad = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int L = seqlens[b] > 0 ? seqlens[b] : 0;
+    for (int t = 0; t < s_new; ++t) {
+      const long long pos = (long long)L + t;
+      if (pos >= (long long)max_pages * page_size) {
+        bad = 1;
+        continue;
+      }
+      const int page = block_table[(size_t)b * max_pages + (size_t)(pos / page_size)];
+      if (page < 0 || page >= num_pages) {
+        bad = 1;
+        continue;
+      }
+      for (int g = 0; g < h_kv; ++g) {
+        const uint16_t* src = new_kv + (((size_t)b * s_new + t) * h_kv + g) * (size_t)d;
+        uint16_t* dst =
+            kvcache + (((size_t)page * page_size + (size_t)(pos % page_size)) * h_kv + g) * (size_t)d;
+        memcpy(dst, src, (size_t)d * sizeof(uint16_t));
+      }
+    }
+  }
+  return bad ? -1 : 0;
+}

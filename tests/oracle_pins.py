@@ -237,6 +237,73 @@ def pin_combine_closed_form(ora):
     _close(l, math.log(4.0), what="combine lse 1:3")
 
 
+def _gather_rows(kvcache, block_table, b, lo, hi):
+    """Rows [lo, hi) of sequence b, gathered through the block table with numpy."""
+    page = kvcache.shape[1]
+    t = np.arange(lo, hi)
+    return kvcache[block_table[b][t // page], t % page]
+
+
+def pin_append_readback(ora):
+    # new rows read back through the block table; every other byte unchanged;
+    # a page boundary is crossed (62 + 5) and one sequence starts empty
+    rng = np.random.default_rng(21)
+    lens = np.array([62, 0, 130], dtype=np.int32)
+    s_new, h_kv, page = 5, 2, 64
+    need = (lens + s_new + page - 1) // page          # pages per sequence after the append
+    pool = int(need.sum()) + 3
+    perm = rng.permutation(pool).astype(np.int32)
+    bt = np.zeros((3, int(need.max()) + 1), dtype=np.int32)
+    k = 0
+    for b in range(3):
+        bt[b, :need[b]] = perm[k:k + need[b]]
+        k += int(need[b])
+    kv = rng.integers(0, 1 << 16, size=(pool, page, h_kv, W.D_QK), dtype=np.uint16)
+    new = rng.integers(0, 1 << 16, size=(3, s_new, h_kv, W.D_QK), dtype=np.uint16)
+    out, ok = ora.append_kvcache(new, bt, lens, kv)
+    assert ok
+    touched = np.zeros(kv.shape[:2], dtype=bool)
+    for b in range(3):
+        L = int(lens[b])
+        assert np.array_equal(_gather_rows(out, bt, b, L, L + s_new), new[b]), f"sequence {b}"
+        t = np.arange(L, L + s_new)
+        touched[bt[b][t // page], t % page] = True
+    assert np.array_equal(out[~touched], kv[~touched]), "rows outside the append changed"
+
+
+def pin_append_then_decode(ora):
+    # truncate a sequence by s_new tokens (garbage in their rows), append the true
+    # rows back: the cache is restored bit for bit and so is the decode
+    inp = small_inputs([200, 77], h_q=4, seed=22)
+    s_new = 3
+    L_full = inp["cache_seqlens"].copy()
+    L_prev = L_full - s_new
+    new = np.stack([_gather_rows(inp["kvcache"], inp["block_table"], b, int(L_prev[b]), int(L_full[b]))
+                    for b in range(2)])
+    damaged = inp["kvcache"].copy()
+    rng = np.random.default_rng(22)
+    for b in range(2):
+        t = np.arange(int(L_prev[b]), int(L_full[b]))
+        damaged[inp["block_table"][b][t // 64], t % 64] = rng.integers(0, 1 << 16, size=(s_new, 1, W.D_QK))
+    out, ok = ora.append_kvcache(new, inp["block_table"], L_prev, damaged)
+    assert ok and np.array_equal(out, inp["kvcache"]), "append did not restore the cache"
+    o1, l1 = _run(ora, inp)
+    o2, l2 = _run(ora, dict(inp, kvcache=out))
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def pin_append_overflow(ora):
+    # a position past the block table is rejected and writes nothing
+    inp = small_inputs([120], h_q=2, seed=23)
+    bt = inp["block_table"][:, :2].copy()  # room for 128 tokens
+    new = np.full((1, 10, 1, W.D_QK), 7, dtype=np.uint16)
+    out, ok = ora.append_kvcache(new, bt, inp["cache_seqlens"], inp["kvcache"])
+    assert not ok
+    got = _gather_rows(out, bt, 0, 120, 128)
+    assert np.all(got == 7), "rows that fit must still be written"
+
+
 ALL_PINS = [pin_bruteforce, pin_single_token, pin_equal_values, pin_page_permutation,
             pin_lse_extended, pin_zero_scale, pin_causal_reduction, pin_split_merge,
-            pin_empty_rows, pin_combine_closed_form]
+            pin_empty_rows, pin_combine_closed_form, pin_append_readback, pin_append_then_decode,
+            pin_append_overflow]

@@ -26,6 +26,10 @@ MUTANTS = {
     "merge_sign": ("const double w = exp(part_lse[k] - total);",
                    "const double w = exp(total - part_lse[k]);"),
     "rope_dims_dropped": ("for (int c = 0; c < d; ++c) acc +=", "for (int c = 0; c < dv; ++c) acc +="),
+    "append_position": ("const long long pos = (long long)L + t;", "const long long pos = (long long)L + t + 1;"),
+    "append_slot": ("(size_t)(pos % page_size)", "(size_t)((pos + 63) % page_size)"),
+    "append_head": ("uint16_t* dst =\n            kvcache + (((size_t)page * page_size + (size_t)(pos % page_size)) * h_kv + g)",
+                    "uint16_t* dst =\n            kvcache + (((size_t)page * page_size + (size_t)(pos % page_size)) * h_kv + 0)"),
 }
 
 
