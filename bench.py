@@ -464,6 +464,52 @@ def bench_reference(args):
     }
 
 
+def bench_append(args):
+    """The cache append (mla_append_kvcache), timed with CUDA events per launch on
+    two shapes: one decode step (64 sequences x 1 new token) and a 1024-token
+    prefill into 64 sequences.  HBM-bound: 2 x 1152 bytes per (token, KV head)."""
+    import torch
+    import paged_mla_attention_b200 as pm
+    peaks, _ = load_peaks()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    rng = np.random.default_rng(7)
+    out = []
+    for name, batch, s_new, L0 in (("decode step", 64, 1, 4096), ("prefill 1024", 64, 1024, 0)):
+        pages_per = (L0 + s_new + 63) // 64
+        pool = batch * pages_per
+        bt = torch.from_numpy(rng.permutation(pool).astype(np.int32).reshape(batch, pages_per)).to(dev)
+        kv = torch.empty((pool, 64, 1, W.D_QK), dtype=torch.bfloat16, device=dev)
+        new = torch.randn((batch, s_new, 1, W.D_QK), device=dev).to(torch.bfloat16)
+        lens = torch.full((batch,), L0, dtype=torch.int32, device=dev)
+        stream = torch.cuda.Stream(dev)
+        with torch.cuda.stream(stream):
+            for _ in range(max(args.warmup, 3)):
+                pm.append_kvcache(new, bt, lens, kv)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()            # one launch per replay, no host overhead inside
+        with torch.cuda.graph(g, stream=stream):
+            pm.append_kvcache(new, bt, lens, kv)
+        g.replay()
+        torch.cuda.synchronize(dev)
+        K = max(args.steps, 10)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+        ev[0].record()
+        for k in range(K):
+            g.replay()
+            ev[k + 1].record()
+        torch.cuda.synchronize(dev)
+        if pm.device_error():
+            raise RuntimeError("device error in the append bench")
+        us = float(np.mean([ev[k].elapsed_time(ev[k + 1]) for k in range(K)])) * 1e3
+        nbytes = 2 * batch * s_new * W.D_QK * 2
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out.append({"shape": f"{name}: batch {batch} x {s_new} tokens, h_kv 1", "us_per_call": round(us, 3),
+                    "bytes": nbytes, "achieved_gbs": round(gbs, 1), "frac_of_hbm_peak": round(gbs / peaks["hbm_gbs"], 4)})
+    return {"metric": "KV-cache append GB/s (read new rows + write cache rows)", "append": out,
+            "n_gpus": 1, "steps": max(args.steps, 10)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -481,6 +527,8 @@ def main():
     ap.add_argument("--no-spot-check", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="plain launches only (warm-up + steps), for ncu; prints one short line")
+    ap.add_argument("--append", action="store_true",
+                    help="time the cache append kernel instead (one JSON line)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per decode call from an ncu capture of the same kernels")
     args = ap.parse_args()
@@ -493,6 +541,10 @@ def main():
         if rank != 0:
             return
         print(json.dumps(bench_reference(args)), flush=True)
+        return
+    if args.append:
+        if rank == 0:
+            print(json.dumps(bench_append(args)), flush=True)
         return
 
     if world > 1:

@@ -51,6 +51,7 @@ extern "C" {
 #define PMLA_ERR_CUDA (-4)         /* a CUDA runtime / driver call or launch failed    */
 #define PMLA_ERR_WORKSPACE (-5)    /* workspace pointer missing or too small           */
 #define PMLA_ERR_DEVICE (-6)       /* a kernel reported an error (see below)           */
+#define PMLA_ERR_EXHAUSTED (-7)    /* the page pool has fewer free pages than asked    */
 
 #define PMLA_PAGE_SIZE 64     /* tokens per KV page                                  */
 #define PMLA_HEAD_DIM 576     /* q / k width: 512 latent (c^KV) + 64 RoPE (k^R)      */
@@ -193,6 +194,64 @@ PMLA_API int mla_decode_with_kvcache_noalloc(const uint16_t* q, const uint16_t* 
                                              const int32_t* num_splits, int causal,
                                              float softmax_scale, uint16_t* o, float* lse,
                                              void* stream);
+
+/*
+ * Append of new tokens to the paged cache (the write side of the paged layout
+ * of the FlashMLA overview, section 4.2(1); the pages describe the cache but
+ * give no call for this, so the signature is ours).  For every sequence b and
+ * new token t < s_new, row t of new_kv is copied to position
+ * cache_seqlens[b] + t of the sequence: page block_table[b][pos / 64], slot
+ * pos % 64, for every KV head.  Decode with cache_seqlens[b] + s_new afterwards.
+ *
+ *   new_kv        bf16 [batch][s_new][h_kv][576], device, 16-byte aligned.
+ *   block_table   int32 [batch][max_pages_per_seq], device: must already hold
+ *                 pages for positions up to cache_seqlens[b] + s_new - 1.
+ *   cache_seqlens int32 [batch], device: lengths before the append (not changed).
+ *   kvcache       bf16 [num_pages][64][h_kv][576], device, written in place.
+ *   new_seqlens   int32 [batch], device, out, optional (NULL): cache_seqlens + s_new.
+ * Runs as one kernel on `stream` (one warp per row, HBM-bound).  A row past the
+ * block table or with a page id outside [0, num_pages) is skipped and recorded
+ * in the device error word (pmla_device_error()).
+ * Errors: INVALID_ARG, UNSUPPORTED (d != 576), ALIGNMENT, CUDA.
+ */
+PMLA_API int mla_append_kvcache(const uint16_t* new_kv, const int32_t* block_table,
+                                const int32_t* cache_seqlens, int batch, int s_new, int h_kv,
+                                int d, uint16_t* kvcache, int num_pages, int max_pages_per_seq,
+                                int32_t* new_seqlens, void* stream);
+
+/*
+ * Page pool for the paged cache (host memory only, no GPU work).  The FlashMLA
+ * overview (section 4.2(1)) describes fixed 64-token physical pages handed to
+ * sequences through block_table; it gives no allocator, so this API is ours.
+ * Page ids are 0..num_pages-1, i.e. indices into the kvcache's first dimension.
+ * Every call is all-or-nothing (on an error the pool is unchanged) and calls on
+ * one pool are serialised internally.
+ *
+ *   pmla_page_pool_create(num_pages, &pool)        -> OK, INVALID_ARG
+ *   pmla_page_pool_destroy(pool)                   frees the pool object
+ *   pmla_page_pool_num_free(pool)                  -> free pages (>= 0) or INVALID_ARG
+ *   pmla_page_pool_alloc(pool, n, pages_out[n])    -> OK, EXHAUSTED (fewer than n free)
+ *   pmla_page_pool_free(pool, n, pages[n])         -> OK, INVALID_ARG (an id out of range,
+ *                                                     not allocated, or repeated)
+ *   pmla_page_pool_grow_sequence(pool, row, max_pages, cur_len, new_len)
+ *       allocates pages for a sequence growing from cur_len to new_len tokens
+ *       into block-table row entries ceil(cur_len/64) .. ceil(new_len/64)-1
+ *       -> OK, EXHAUSTED, INVALID_ARG (new_len < cur_len or past max_pages)
+ *   pmla_page_pool_release_sequence(pool, row, len) frees the ceil(len/64)
+ *       pages of a sequence of len tokens -> OK, INVALID_ARG
+ * `row`, `pages` and `pages_out` are host int32 arrays owned by the caller;
+ * copy block tables to the device for mla_decode_with_kvcache.
+ */
+typedef struct pmla_page_pool pmla_page_pool;
+PMLA_API int pmla_page_pool_create(int num_pages, pmla_page_pool** out);
+PMLA_API void pmla_page_pool_destroy(pmla_page_pool* pool);
+PMLA_API int pmla_page_pool_num_free(pmla_page_pool* pool);
+PMLA_API int pmla_page_pool_alloc(pmla_page_pool* pool, int n, int32_t* pages_out);
+PMLA_API int pmla_page_pool_free(pmla_page_pool* pool, int n, const int32_t* pages);
+PMLA_API int pmla_page_pool_grow_sequence(pmla_page_pool* pool, int32_t* block_table_row,
+                                          int max_pages, int cur_len, int new_len);
+PMLA_API int pmla_page_pool_release_sequence(pmla_page_pool* pool, const int32_t* block_table_row,
+                                             int len);
 
 /*
  * Reads and clears the device error word of the current device (synchronises

@@ -21,6 +21,7 @@ import math
 import os
 from typing import Optional, Tuple
 
+import numpy as np
 import torch
 
 __all__ = ["get_mla_metadata", "flash_mla_with_kvcache", "device_error", "library", "LIB_PATH",
@@ -36,7 +37,7 @@ METADATA_INTS = 8
 DEFAULT_SOFTMAX_SCALE = 1.0 / math.sqrt(192.0)
 
 ERRORS = {-1: "invalid argument", -2: "unsupported", -3: "alignment", -4: "CUDA error",
-          -5: "workspace", -6: "device error"}
+          -5: "workspace", -6: "device error", -7: "page pool exhausted"}
 
 
 class PmlaError(RuntimeError):
@@ -59,6 +60,22 @@ def _load() -> ctypes.CDLL:
         fn = getattr(lib, name)
         fn.argtypes = [P, P, P, P] + [I] * 8 + [P, I, P, I, ctypes.c_float, P, P, P, SZ, P]
         fn.restype = I
+    lib.pmla_page_pool_create.argtypes = [I, ctypes.POINTER(P)]
+    lib.pmla_page_pool_create.restype = I
+    lib.pmla_page_pool_destroy.argtypes = [P]
+    lib.pmla_page_pool_destroy.restype = None
+    lib.pmla_page_pool_num_free.argtypes = [P]
+    lib.pmla_page_pool_num_free.restype = I
+    lib.pmla_page_pool_alloc.argtypes = [P, I, P]
+    lib.pmla_page_pool_alloc.restype = I
+    lib.pmla_page_pool_free.argtypes = [P, I, P]
+    lib.pmla_page_pool_free.restype = I
+    lib.pmla_page_pool_grow_sequence.argtypes = [P, P, I, I, I]
+    lib.pmla_page_pool_grow_sequence.restype = I
+    lib.pmla_page_pool_release_sequence.argtypes = [P, P, I]
+    lib.pmla_page_pool_release_sequence.restype = I
+    lib.mla_append_kvcache.argtypes = [P, P, P, I, I, I, I, P, I, I, P, P]
+    lib.mla_append_kvcache.restype = I
     lib.pmla_device_error.argtypes = []
     lib.pmla_device_error.restype = I
     lib.pmla_last_error.argtypes = []
@@ -199,6 +216,92 @@ def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: 
             _ptr(num_splits), int(bool(causal)), scale, _ptr(o), _ptr(lse), _ptr(workspace),
             workspace.numel(), _stream_ptr(dev)))
     return o, lse
+
+
+def append_kvcache(new_kv: torch.Tensor, block_table: torch.Tensor, cache_seqlens: torch.Tensor,
+                   kvcache: torch.Tensor, new_seqlens: Optional[torch.Tensor] = None) -> Optional[torch.Tensor]:
+    """Write new tokens into the paged cache in place (mla_append_kvcache).
+
+    new_kv      bf16 [batch, s_new, h_kv, 576]
+    block_table int32 [batch, max_pages] (pages already assigned for the new positions)
+    cache_seqlens int32 [batch], lengths before the append
+    kvcache     bf16 [num_pages, 64, h_kv, 576], modified in place
+    new_seqlens optional int32 [batch] out: cache_seqlens + s_new (returned).
+    """
+    _need(new_kv, "new_kv", torch.bfloat16, 4)
+    _need(kvcache, "kvcache", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(cache_seqlens, "cache_seqlens", torch.int32, 1)
+    batch, s_new, h_kv, d = new_kv.shape
+    num_pages, page, h_kv2, d2 = kvcache.shape
+    if page != PAGE_SIZE or h_kv2 != h_kv or d2 != d:
+        raise ValueError(f"kvcache {tuple(kvcache.shape)} does not match new_kv {tuple(new_kv.shape)}")
+    if block_table.shape[0] != batch or cache_seqlens.shape[0] != batch:
+        raise ValueError("batch size mismatch between new_kv, block_table and cache_seqlens")
+    dev = new_kv.device
+    for name, t in (("kvcache", kvcache), ("block_table", block_table), ("cache_seqlens", cache_seqlens)):
+        if t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, new_kv on {dev}")
+    if new_seqlens is not None:
+        _need(new_seqlens, "new_seqlens", torch.int32, 1)
+    with torch.cuda.device(dev):
+        _check(library.mla_append_kvcache(_ptr(new_kv), _ptr(block_table), _ptr(cache_seqlens), batch, s_new,
+                                          h_kv, d, _ptr(kvcache), num_pages, block_table.shape[1],
+                                          _ptr(new_seqlens) if new_seqlens is not None else None,
+                                          _stream_ptr(dev)))
+    return new_seqlens
+
+
+class PagePool:
+    """Host-side pool of 64-token cache pages (the pmla_page_pool_* C calls).
+
+    Page ids index the kvcache's first dimension.  ``grow`` / ``release`` keep a
+    sequence's block-table row (a host int32 numpy array) in step with its
+    length; copy the table to the device for the decode call.
+    """
+
+    def __init__(self, num_pages: int):
+        h = ctypes.c_void_p()
+        _check(library.pmla_page_pool_create(int(num_pages), ctypes.byref(h)))
+        self._h = h
+        self.num_pages = int(num_pages)
+
+    def close(self) -> None:
+        if self._h:
+            library.pmla_page_pool_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def num_free(self) -> int:
+        n = library.pmla_page_pool_num_free(self._h)
+        if n < 0:
+            raise PmlaError(n, "pmla_page_pool_num_free failed")
+        return int(n)
+
+    def alloc(self, n: int) -> "np.ndarray":
+        out = np.empty(int(n), dtype=np.int32)
+        _check(library.pmla_page_pool_alloc(self._h, int(n), out.ctypes.data_as(ctypes.c_void_p)))
+        return out
+
+    def free(self, pages) -> None:
+        a = np.ascontiguousarray(pages, dtype=np.int32)
+        _check(library.pmla_page_pool_free(self._h, a.size, a.ctypes.data_as(ctypes.c_void_p)))
+
+    def grow(self, row: "np.ndarray", cur_len: int, new_len: int) -> None:
+        if row.dtype != np.int32 or not row.flags["C_CONTIGUOUS"]:
+            raise ValueError("block-table row must be a contiguous int32 numpy array")
+        _check(library.pmla_page_pool_grow_sequence(self._h, row.ctypes.data_as(ctypes.c_void_p), row.size,
+                                                    int(cur_len), int(new_len)))
+
+    def release(self, row: "np.ndarray", length: int) -> None:
+        a = np.ascontiguousarray(row, dtype=np.int32)
+        _check(library.pmla_page_pool_release_sequence(self._h, a.ctypes.data_as(ctypes.c_void_p), int(length)))
 
 
 def workspace_bytes(batch: int, s_q: int, h_q: int, h_kv: int) -> int:

@@ -364,6 +364,44 @@ int mla_decode_with_kvcache(PMLA_DECODE_PARAMS) {
 int mla_decode_splits(PMLA_DECODE_PARAMS) { return decode_impl(PMLA_DECODE_ARGS, kStageDecode); }
 int mla_merge_splits(PMLA_DECODE_PARAMS) { return decode_impl(PMLA_DECODE_ARGS, kStageMerge); }
 
+int mla_append_kvcache(const uint16_t* new_kv, const int32_t* block_table,
+                       const int32_t* cache_seqlens, int batch, int s_new, int h_kv, int d,
+                       uint16_t* kvcache, int num_pages, int max_pages_per_seq,
+                       int32_t* new_seqlens, void* stream) {
+  g_last_error.clear();
+  if (d != PMLA_HEAD_DIM) return fail(PMLA_ERR_UNSUPPORTED, "head dim must be d=576 (got %d)", d);
+  if (batch < 0 || batch > 65535 || s_new < 0 || h_kv < 1 || h_kv > 65535)
+    return fail(PMLA_ERR_INVALID_ARG, "bad shape batch=%d s_new=%d h_kv=%d", batch, s_new, h_kv);
+  if (num_pages < 1 || max_pages_per_seq < 1)
+    return fail(PMLA_ERR_INVALID_ARG, "num_pages and max_pages_per_seq must be >= 1");
+  if ((long long)batch * s_new * h_kv > (1ll << 40))
+    return fail(PMLA_ERR_UNSUPPORTED, "too many rows");
+  if ((long long)batch * s_new == 0) return PMLA_OK;
+  if (!new_kv || !block_table || !cache_seqlens || !kvcache)
+    return fail(PMLA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(new_kv) || !aligned16(kvcache))
+    return fail(PMLA_ERR_ALIGNMENT, "new_kv and kvcache must be 16-byte aligned");
+  int dev;
+  DeviceInfo* info;
+  int rc = device_setup(&dev, &info);
+  if (rc) return rc;
+  pmla::AppendParams a;
+  a.new_kv = new_kv;
+  a.block_table = block_table;
+  a.seqlens = cache_seqlens;
+  a.kvcache = kvcache;
+  a.new_seqlens = new_seqlens;
+  a.err = info->err_ptr;
+  a.batch = batch;
+  a.s_new = s_new;
+  a.h_kv = h_kv;
+  a.max_pages = max_pages_per_seq;
+  a.num_pages = num_pages;
+  cudaError_t e = pmla::launch_append(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "append kernel launch");
+  return PMLA_OK;
+}
+
 int pmla_device_error(void) {
   int dev;
   DeviceInfo* info;

@@ -26,6 +26,7 @@ enum DeviceError : int {
   kErrNone = 0,
   kErrBadSmemAlign = 1,
   kErrBadPage = 2,
+  kErrBadAppend = 3,   // an appended token lies past the sequence's block table
   kErrWaitBase = 100,  // + the id of the wait that gave up
 };
 
@@ -60,6 +61,16 @@ struct CombineParams {
   int batch, s_q, h_q, h_kv, hpk, R, n_rg, num_parts;
 };
 
+struct AppendParams {
+  const uint16_t* new_kv;       // [b][s_new][h_kv][576]
+  const int32_t* block_table;   // [b][max_pages]
+  const int32_t* seqlens;       // [b], lengths before the append
+  uint16_t* kvcache;            // [num_pages][64][h_kv][576]
+  int32_t* new_seqlens;         // [b] or null: seqlens + s_new
+  int* err;                     // device error word
+  int batch, s_new, h_kv, max_pages, num_pages;
+};
+
 // Workspace layout of one decode call: split partials o (chunk-major fp32),
 // their lse, and the per-(sequence, KV head, row group) completion counters the
 // merge kernel waits on.  Returns the total size.
@@ -76,6 +87,7 @@ int decode_max_active_clusters(int device, int* out);
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, const CUtensorMap& tmap_q,
                           const CUtensorMap& tmap_v, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
+cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 size_t decode_smem_bytes();
 
 // Records the message pmla_last_error() returns on this host thread.

@@ -78,3 +78,34 @@ def test_metadata_rejects_bad_arguments(lib):
     assert f(0x1000, 4, 0, 1, 0x2000, 4, 0x3000, None) == -1
     assert f(0x1000, 4, 128, 1, None, 4, 0x3000, None) == -1
     assert f(0x1000, 4, 128, 1, 0x2000, 0, 0x3000, None) == -1
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=512), -2),            # UNSUPPORTED: only d = 576 rows
+    (dict(s_new=-1), -1),         # INVALID_ARG
+    (dict(h_kv=0), -1),
+    (dict(num_pages=0), -1),
+    (dict(new_kv=0x1008), -3),    # ALIGNMENT: new_kv not 16-byte aligned
+    (dict(kvcache=0), -1),        # null pointer
+])
+def test_append_rejects_bad_arguments(lib, kw, code):
+    args = dict(new_kv=0x1000, block_table=0x2000, cache_seqlens=0x3000, batch=2, s_new=1, h_kv=1,
+                d=576, kvcache=0x4000, num_pages=8, max_pages=2, new_seqlens=None)
+    args.update(kw)
+    f = lib.mla_append_kvcache
+    P, I = ctypes.c_void_p, ctypes.c_int
+    f.argtypes = [P, P, P, I, I, I, I, P, I, I, P, P]
+    f.restype = I
+    rc = f(args["new_kv"], args["block_table"], args["cache_seqlens"], args["batch"], args["s_new"],
+           args["h_kv"], args["d"], args["kvcache"], args["num_pages"], args["max_pages"],
+           args["new_seqlens"], None)
+    assert rc == code
+
+
+def test_append_with_nothing_to_write_is_a_no_op(lib):
+    f = lib.mla_append_kvcache
+    P, I = ctypes.c_void_p, ctypes.c_int
+    f.argtypes = [P, P, P, I, I, I, I, P, I, I, P, P]
+    f.restype = I
+    assert f(None, None, None, 0, 1, 1, 576, None, 8, 2, None, None) == 0   # empty batch
+    assert f(None, None, None, 4, 0, 1, 576, None, 8, 2, None, None) == 0   # no new tokens
