@@ -55,6 +55,8 @@ class OracleLib:
         lib.oracle_num_threads.restype = I
         lib.oracle_append_kvcache.argtypes = [P, P, P] + [I] * 7 + [P]
         lib.oracle_append_kvcache.restype = I
+        lib.oracle_mla_decode_unabsorbed.argtypes = [P] * 7 + [I] * 6 + [ctypes.c_double, P, P, I]
+        lib.oracle_mla_decode_unabsorbed.restype = I
         self.lib = lib
         self.path = path
 
@@ -118,6 +120,32 @@ class OracleLib:
         rc = self.lib.oracle_append_kvcache(_ptr(new_kv), _ptr(block_table), _ptr(cache_seqlens), b,
                                             s_new, h_kv, d, page, block_table.shape[1], pages, _ptr(out))
         return out, rc == 0
+
+    def mla_decode_unabsorbed(self, q_nope: np.ndarray, q_rope: np.ndarray, w_uk: np.ndarray,
+                              w_uv: np.ndarray, kvcache: np.ndarray, block_table: np.ndarray,
+                              cache_seqlens: np.ndarray, causal: bool,
+                              softmax_scale: float) -> Tuple[np.ndarray, np.ndarray]:
+        """Per-head up-projected attention (h_kv = 1): q_nope [b][s_q][h][128], q_rope
+        [b][s_q][h][64], w_uk and w_uv [h][128][512] (float64); kvcache uint16 bf16 bits.
+        Returns (o float64 [b][s_q][h][128], lse float64 [b][h][s_q])."""
+        q_nope = np.ascontiguousarray(q_nope, dtype=np.float64)
+        q_rope = np.ascontiguousarray(q_rope, dtype=np.float64)
+        w_uk = np.ascontiguousarray(w_uk, dtype=np.float64)
+        w_uv = np.ascontiguousarray(w_uv, dtype=np.float64)
+        kvcache = np.ascontiguousarray(kvcache, dtype=np.uint16)
+        block_table = np.ascontiguousarray(block_table, dtype=np.int32)
+        cache_seqlens = np.ascontiguousarray(cache_seqlens, dtype=np.int32)
+        b, s_q, h, _ = q_nope.shape
+        assert kvcache.shape[2] == 1 and kvcache.shape[3] == 576
+        o = np.zeros((b, s_q, h, 128), dtype=np.float64)
+        lse = np.zeros((b, h, s_q), dtype=np.float64)
+        rc = self.lib.oracle_mla_decode_unabsorbed(
+            _ptr(q_nope), _ptr(q_rope), _ptr(w_uk), _ptr(w_uv), _ptr(kvcache), _ptr(block_table),
+            _ptr(cache_seqlens), b, s_q, h, kvcache.shape[1], block_table.shape[1], int(bool(causal)),
+            float(softmax_scale), _ptr(o), _ptr(lse), 0)
+        if rc != 0:
+            raise ValueError("oracle_mla_decode_unabsorbed rejected its arguments")
+        return o, lse
 
     def decode_inputs(self, inp: dict, nthreads: int = 0, **kw) -> Tuple[np.ndarray, np.ndarray]:
         """Run on an input dict from ``mla_workloads.make_inputs``."""

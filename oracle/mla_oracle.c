@@ -205,3 +205,77 @@ int oracle_append_kvcache(const uint16_t* new_kv, const int32_t* block_table,
   }
   return bad ? -1 : 0;
 }
+
+/*
+ * Unabsorbed MLA decode for one KV head (FlashMLA overview, section 2.2): per
+ * query head h the key and value of cached token j are up-projected from the
+ * latent c_j = row[0:512] with per-head matrices
+ *     k^C_{j,h} = W^UK_h c_j   (128),    v_{j,h} = W^UV_h c_j   (128),
+ * with W^UK_h, W^UV_h stored [h][128][512]; the RoPE part k^R_j = row[512:576]
+ * is shared by all heads.  Score_h(j) = scale * (q^C_h . k^C_{j,h} + q^R_h . k^R_j),
+ * o_h = sum_j softmax_j(Score_h) v_{j,h}, lse_h = log sum_j exp(Score_h(j)).
+ * Same masking readings as oracle_mla_decode; h_kv = 1.  q_nope [b][s_q][h_q][128]
+ * and q_rope [b][s_q][h_q][64] are fp64; o [b][s_q][h_q][128], lse [b][h_q][s_q].
+ */
+int oracle_mla_decode_unabsorbed(const double* q_nope, const double* q_rope, const double* w_uk,
+                                 const double* w_uv, const uint16_t* kv, const int32_t* block_table,
+                                 const int32_t* seqlens, int batch, int s_q, int h_q, int page_size,
+                                 int max_pages, int causal, double softmax_scale, double* o,
+                                 double* lse, int nthreads) {
+  const int dn = 128, dr = 64, dc = 512, d = 576, dvo = 128;
+  if (batch < 0 || s_q < 1 || h_q < 1 || page_size < 1) return -1;
+  (void)nthreads;
+  double* s = NULL;
+  double* c = (double*)malloc(sizeof(double) * d);
+  for (int b = 0; b < batch; ++b) {
+    const int L = seqlens[b] > 0 ? seqlens[b] : 0;
+    free(s);
+    s = (double*)malloc(sizeof(double) * (L > 0 ? L : 1));
+    for (int i = 0; i < s_q; ++i) {
+      const int last = causal ? (L - s_q) + i : L - 1;
+      for (int h = 0; h < h_q; ++h) {
+        const double* qn = q_nope + (((size_t)b * s_q + i) * h_q + h) * dn;
+        const double* qr = q_rope + (((size_t)b * s_q + i) * h_q + h) * dr;
+        const double* wk = w_uk + (size_t)h * dn * dc;
+        const double* wv = w_uv + (size_t)h * dvo * dc;
+        double* orow = o + (((size_t)b * s_q + i) * h_q + h) * dvo;
+        for (int c2 = 0; c2 < dvo; ++c2) orow[c2] = 0.0;
+        double* lse_out = lse + ((size_t)b * h_q + h) * s_q + i;
+        if (last < 0) {
+          *lse_out = -INFINITY;
+          continue;
+        }
+        double m = -INFINITY;
+        for (int j = 0; j <= last; ++j) {
+          const uint16_t* row = kv_row(kv, block_table, max_pages, b, j, 0, 1, d, page_size);
+          for (int k = 0; k < d; ++k) c[k] = bf16_to_double(row[k]);
+          double acc = 0.0;
+          for (int r = 0; r < dn; ++r) {  /* k^C_{j,h}[r] = sum_k W^UK_h[r][k] c_j[k] */
+            double t = 0.0;
+            for (int k = 0; k < dc; ++k) t += wk[(size_t)r * dc + k] * c[k];
+            acc += qn[r] * t;
+          }
+          for (int r = 0; r < dr; ++r) acc += qr[r] * c[dc + r];
+          s[j] = softmax_scale * acc;
+          if (s[j] > m) m = s[j];
+        }
+        double z = 0.0;
+        for (int j = 0; j <= last; ++j) z += exp(s[j] - m);
+        for (int j = 0; j <= last; ++j) {
+          const double w = exp(s[j] - m) / z;
+          const uint16_t* row = kv_row(kv, block_table, max_pages, b, j, 0, 1, d, page_size);
+          for (int k = 0; k < dc; ++k) c[k] = bf16_to_double(row[k]);
+          for (int r = 0; r < dvo; ++r) {  /* v_{j,h}[r] = sum_k W^UV_h[r][k] c_j[k] */
+            double t = 0.0;
+            for (int k = 0; k < dc; ++k) t += wv[(size_t)r * dc + k] * c[k];
+            orow[r] += w * t;
+          }
+        }
+        *lse_out = log(z) + m;
+      }
+    }
+  }
+  free(s);
+  free(c);
+  return 0;
+}

@@ -303,7 +303,59 @@ def pin_append_overflow(ora):
     assert np.all(got == 7), "rows that fit must still be written"
 
 
+def _mla_weights(h, seed):
+    rng = np.random.default_rng(seed)
+    w_uk = rng.standard_normal((h, 128, 512)) / math.sqrt(512)
+    w_uv = rng.standard_normal((h, 128, 512)) / math.sqrt(512)
+    return w_uk, w_uv
+
+
+def pin_unabsorbed_bruteforce(ora):
+    # per-head up-projected keys and values, written densely with numpy
+    inp = small_inputs([70, 5], h_q=3, seed=31, s_q=2, causal=True)
+    rng = np.random.default_rng(31)
+    b, s_q, h = 2, 2, 3
+    qn = rng.standard_normal((b, s_q, h, 128))
+    qr = rng.standard_normal((b, s_q, h, 64))
+    w_uk, w_uv = _mla_weights(h, 31)
+    o, lse = ora.mla_decode_unabsorbed(qn, qr, w_uk, w_uv, inp["kvcache"], inp["block_table"],
+                                       inp["cache_seqlens"], True, inp["softmax_scale"])
+    for bb in range(b):
+        L = int(inp["cache_seqlens"][bb])
+        rows = W.bf16_bits_to_f32(_gather_rows(inp["kvcache"], inp["block_table"], bb, 0, L)[:, 0]).astype(np.float64)
+        C, KR = rows[:, :512], rows[:, 512:]
+        for i in range(s_q):
+            last = L - s_q + i
+            for hh in range(h):
+                kC = C[:last + 1] @ w_uk[hh].T
+                v = C[:last + 1] @ w_uv[hh].T
+                sc = inp["softmax_scale"] * (kC @ qn[bb, i, hh] + KR[:last + 1] @ qr[bb, i, hh])
+                m = sc.max()
+                p = np.exp(sc - m)
+                assert np.allclose(o[bb, i, hh], (p / p.sum()) @ v, rtol=0, atol=1e-10)
+                assert abs(lse[bb, hh, i] - (m + math.log(p.sum()))) < 1e-10
+
+
+def pin_unabsorbed_equals_absorbed_route(ora):
+    # W^UK = [I | 0] makes the absorbed query [q^C, 0, ..] exact in bf16, so the latent
+    # decode oracle applies; W^UV times its output must equal the unabsorbed result
+    inp = small_inputs([130, 40], h_q=2, seed=32)
+    b, h = 2, 2
+    q = inp["q"].copy()
+    q[..., 128:512] = 0                    # latent query beyond the first 128 dims
+    qn = W.bf16_bits_to_f32(q[..., :128]).astype(np.float64)
+    qr = W.bf16_bits_to_f32(q[..., 512:]).astype(np.float64)
+    w_uk = np.zeros((h, 128, 512))
+    w_uk[:, np.arange(128), np.arange(128)] = 1.0
+    _, w_uv = _mla_weights(h, 32)
+    o_lat, lse_lat = _run(ora, dict(inp, q=q))
+    o, lse = ora.mla_decode_unabsorbed(qn, qr, w_uk, w_uv, inp["kvcache"], inp["block_table"],
+                                       inp["cache_seqlens"], False, inp["softmax_scale"])
+    assert np.allclose(o, np.einsum("bshk,hrk->bshr", o_lat, w_uv), rtol=0, atol=1e-10)
+    assert np.allclose(lse, lse_lat, rtol=0, atol=1e-10)
+
+
 ALL_PINS = [pin_bruteforce, pin_single_token, pin_equal_values, pin_page_permutation,
             pin_lse_extended, pin_zero_scale, pin_causal_reduction, pin_split_merge,
             pin_empty_rows, pin_combine_closed_form, pin_append_readback, pin_append_then_decode,
-            pin_append_overflow]
+            pin_append_overflow, pin_unabsorbed_bruteforce, pin_unabsorbed_equals_absorbed_route]

@@ -28,6 +28,9 @@ MUTANTS = {
     "rope_dims_dropped": ("for (int c = 0; c < d; ++c) acc +=", "for (int c = 0; c < dv; ++c) acc +="),
     "append_position": ("const long long pos = (long long)L + t;", "const long long pos = (long long)L + t + 1;"),
     "append_slot": ("(size_t)(pos % page_size)", "(size_t)((pos + 63) % page_size)"),
+    "unabsorbed_wv_transposed": ("t += wv[(size_t)r * dc + k] * c[k];", "t += wv[(size_t)k * dvo + r] * c[k];"),
+    "unabsorbed_rope_dropped": ("for (int r = 0; r < dr; ++r) acc += qr[r] * c[dc + r];",
+                                "for (int r = 0; r < dr; ++r) acc += 0.0 * qr[r] * c[dc + r];"),
     "append_head": ("uint16_t* dst =\n            kvcache + (((size_t)page * page_size + (size_t)(pos % page_size)) * h_kv + g)",
                     "uint16_t* dst =\n            kvcache + (((size_t)page * page_size + (size_t)(pos % page_size)) * h_kv + 0)"),
 }
