@@ -510,6 +510,61 @@ def bench_append(args):
             "n_gpus": 1, "steps": max(args.steps, 10)}
 
 
+def bench_proj(args):
+    """The absorbed projections (mla_absorb_query before the decode, mla_project_output
+    after it), timed with CUDA events per launch at three token counts with 128 heads.
+    Bytes: activations in and out plus each head's 128 x 512 bf16 weight matrix (read
+    once per 128-token tile); FLOPs 2 x 128 x 512 per (token, head)."""
+    import torch
+    import paged_mla_attention_b200 as pm
+    peaks, _ = load_peaks()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    H = 128
+    out = []
+    for T in (64, 128, 1024):
+        qn = torch.randn((T, H, 128), device=dev).to(torch.bfloat16)
+        qr = torch.randn((T, H, 64), device=dev).to(torch.bfloat16)
+        ol = torch.randn((T, H, 512), device=dev).to(torch.bfloat16)
+        w_uk = (torch.randn((H, 128, 512), device=dev) / 11.3).to(torch.bfloat16)
+        w_uv = (torch.randn((H, 128, 512), device=dev) / 22.6).to(torch.bfloat16)
+        q = torch.empty((T, H, 576), dtype=torch.bfloat16, device=dev)
+        o = torch.empty((T, H, 128), dtype=torch.bfloat16, device=dev)
+        tiles = (T + 127) // 128
+        wbytes = H * 128 * 512 * 2 * tiles
+        for name, fn, nbytes in (
+                ("absorb_query", lambda: pm.absorb_query(qn, qr, w_uk, out=q), T * H * (192 + 576) * 2 + wbytes),
+                ("project_output", lambda: pm.project_output(ol, w_uv, out=o), T * H * (512 + 128) * 2 + wbytes)):
+            stream = torch.cuda.Stream(dev)
+            with torch.cuda.stream(stream):
+                for _ in range(max(args.warmup, 3)):
+                    fn()
+            torch.cuda.synchronize(dev)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+            g.replay()
+            torch.cuda.synchronize(dev)
+            K = max(args.steps, 10)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+            ev[0].record()
+            for k in range(K):
+                g.replay()
+                ev[k + 1].record()
+            torch.cuda.synchronize(dev)
+            if pm.device_error():
+                raise RuntimeError("device error in the projection bench")
+            us = float(np.mean([ev[k].elapsed_time(ev[k + 1]) for k in range(K)])) * 1e3
+            gbs = nbytes / (us * 1e-6) / 1e9
+            tfs = 2.0 * T * H * 128 * 512 / (us * 1e-6) / 1e12
+            out.append({"kernel": name, "tokens": T, "heads": H, "us_per_call": round(us, 3),
+                        "bytes": nbytes, "achieved_gbs": round(gbs, 1),
+                        "frac_of_hbm_peak": round(gbs / peaks["hbm_gbs"], 4),
+                        "tflops": round(tfs, 2), "frac_of_bf16_peak": round(tfs / peaks["bf16_tflops"], 4)})
+    return {"metric": "absorbed projection kernels (us per call; HBM and tensor fractions)", "proj": out,
+            "n_gpus": 1, "steps": max(args.steps, 10)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -529,6 +584,8 @@ def main():
                     help="plain launches only (warm-up + steps), for ncu; prints one short line")
     ap.add_argument("--append", action="store_true",
                     help="time the cache append kernel instead (one JSON line)")
+    ap.add_argument("--proj", action="store_true",
+                    help="time the absorbed projection kernels instead (one JSON line)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per decode call from an ncu capture of the same kernels")
     args = ap.parse_args()
@@ -541,6 +598,10 @@ def main():
         if rank != 0:
             return
         print(json.dumps(bench_reference(args)), flush=True)
+        return
+    if args.proj:
+        if rank == 0:
+            print(json.dumps(bench_proj(args)), flush=True)
         return
     if args.append:
         if rank == 0:

@@ -254,6 +254,27 @@ PMLA_API int pmla_page_pool_release_sequence(pmla_page_pool* pool, const int32_t
                                              int len);
 
 /*
+ * Absorbed MLA projections around the latent decode (FlashMLA overview,
+ * section 2.2, "matrix absorption"): per query head h, with W^UK_h and W^UV_h
+ * the key and value up-projections (128 x 512 each, stored [h][128][512], bf16),
+ *   mla_absorb_query:   q[t][h] = [ W^UK_h^T q_nope[t][h] (512) ; q_rope[t][h] (64) ]
+ *   mla_project_output: o[t][h] = W^UV_h o_latent[t][h]           (128)
+ * so that decoding q against the latent cache and projecting its output equals
+ * attention with the up-projected per-head keys and values.  t runs over the
+ * `tokens` query tokens (batch * s_q); one KV head.  Tensor-core GEMMs with
+ * fp32 accumulation, bf16 results; the pages give no call for these steps, so
+ * the signatures are ours.
+ *   q_nope [tokens][heads][128], q_rope [tokens][heads][64], q_out [tokens][heads][576]
+ *   o_latent [tokens][heads][512], o_out [tokens][heads][128]
+ * Inputs 16-byte aligned, outputs 32-byte aligned, all device memory.
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA.
+ */
+PMLA_API int mla_absorb_query(const uint16_t* q_nope, const uint16_t* q_rope, const uint16_t* w_uk,
+                              int tokens, int heads, uint16_t* q_out, void* stream);
+PMLA_API int mla_project_output(const uint16_t* o_latent, const uint16_t* w_uv, int tokens, int heads,
+                                uint16_t* o_out, void* stream);
+
+/*
  * Reads and clears the device error word of the current device (synchronises
  * the device).  Returns 0 if no kernel reported an error since the last call,
  * else the kernel's error code (a positive number naming the wait that gave up).

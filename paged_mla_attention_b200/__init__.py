@@ -74,6 +74,10 @@ def _load() -> ctypes.CDLL:
     lib.pmla_page_pool_grow_sequence.restype = I
     lib.pmla_page_pool_release_sequence.argtypes = [P, P, I]
     lib.pmla_page_pool_release_sequence.restype = I
+    lib.mla_absorb_query.argtypes = [P, P, P, I, I, P, P]
+    lib.mla_absorb_query.restype = I
+    lib.mla_project_output.argtypes = [P, P, I, I, P, P]
+    lib.mla_project_output.restype = I
     lib.mla_append_kvcache.argtypes = [P, P, P, I, I, I, I, P, I, I, P, P]
     lib.mla_append_kvcache.restype = I
     lib.pmla_device_error.argtypes = []
@@ -250,6 +254,46 @@ def append_kvcache(new_kv: torch.Tensor, block_table: torch.Tensor, cache_seqlen
                                           _ptr(new_seqlens) if new_seqlens is not None else None,
                                           _stream_ptr(dev)))
     return new_seqlens
+
+
+def absorb_query(q_nope: torch.Tensor, q_rope: torch.Tensor, w_uk: torch.Tensor,
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Absorbed 576-wide query: [W^UK_h^T q_nope (512) ; q_rope (64)] per token and head.
+
+    q_nope bf16 [T, H, 128], q_rope bf16 [T, H, 64], w_uk bf16 [H, 128, 512] -> bf16 [T, H, 576].
+    """
+    _need(q_nope, "q_nope", torch.bfloat16, 3)
+    _need(q_rope, "q_rope", torch.bfloat16, 3)
+    _need(w_uk, "w_uk", torch.bfloat16, 3)
+    T, H, dn = q_nope.shape
+    if dn != 128 or tuple(q_rope.shape) != (T, H, 64) or tuple(w_uk.shape) != (H, 128, 512):
+        raise ValueError("shapes must be q_nope [T,H,128], q_rope [T,H,64], w_uk [H,128,512]")
+    dev = q_nope.device
+    if out is None:
+        out = torch.empty((T, H, 576), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, 3)
+    with torch.cuda.device(dev):
+        _check(library.mla_absorb_query(_ptr(q_nope), _ptr(q_rope), _ptr(w_uk), T, H, _ptr(out),
+                                        _stream_ptr(dev)))
+    return out
+
+
+def project_output(o_latent: torch.Tensor, w_uv: torch.Tensor,
+                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Per-head output W^UV_h o_latent: o_latent bf16 [T, H, 512], w_uv bf16 [H, 128, 512]
+    -> bf16 [T, H, 128]."""
+    _need(o_latent, "o_latent", torch.bfloat16, 3)
+    _need(w_uv, "w_uv", torch.bfloat16, 3)
+    T, H, dc = o_latent.shape
+    if dc != 512 or tuple(w_uv.shape) != (H, 128, 512):
+        raise ValueError("shapes must be o_latent [T,H,512], w_uv [H,128,512]")
+    dev = o_latent.device
+    if out is None:
+        out = torch.empty((T, H, 128), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, 3)
+    with torch.cuda.device(dev):
+        _check(library.mla_project_output(_ptr(o_latent), _ptr(w_uv), T, H, _ptr(out), _stream_ptr(dev)))
+    return out
 
 
 class PagePool:

@@ -16,7 +16,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libpagedmla.so")
-SOURCES = ["api.cu", "sched.cu", "decode.cu", "combine.cu", "noalloc.cu", "append.cu", "pages.cpp"]
+SOURCES = ["api.cu", "sched.cu", "decode.cu", "combine.cu", "noalloc.cu", "append.cu", "proj.cu", "pages.cpp"]
 HEADERS = ["ptx.cuh", "pagedmla_internal.cuh", os.path.join("..", "..", "include", "pagedmla.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -402,6 +402,42 @@ int mla_append_kvcache(const uint16_t* new_kv, const int32_t* block_table,
   return PMLA_OK;
 }
 
+static int proj_call(const uint16_t* a, const uint16_t* rope, const uint16_t* w, int tokens, int heads,
+                     uint16_t* out, void* stream, bool absorb) {
+  g_last_error.clear();
+  if (tokens < 0 || heads < 1 || heads > 65535 || (long long)tokens > (1ll << 31))
+    return fail(PMLA_ERR_INVALID_ARG, "bad shape tokens=%d heads=%d", tokens, heads);
+  if (tokens == 0) return PMLA_OK;
+  if (!a || !w || !out || (absorb && !rope)) return fail(PMLA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(a) || !aligned16(w) || !aligned32(out) || (absorb && !aligned16(rope)))
+    return fail(PMLA_ERR_ALIGNMENT, "inputs must be 16-byte aligned and the output 32-byte aligned");
+  int dev;
+  DeviceInfo* info;
+  int rc = device_setup(&dev, &info);
+  if (rc) return rc;
+  pmla::ProjParams p;
+  p.a = a;
+  p.rope = rope;
+  p.w = w;
+  p.out = out;
+  p.err = info->err_ptr;
+  p.tokens = tokens;
+  p.heads = heads;
+  cudaError_t e = pmla::launch_proj(p, absorb, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e, "projection kernel launch");
+  return PMLA_OK;
+}
+
+int mla_absorb_query(const uint16_t* q_nope, const uint16_t* q_rope, const uint16_t* w_uk, int tokens,
+                     int heads, uint16_t* q_out, void* stream) {
+  return proj_call(q_nope, q_rope, w_uk, tokens, heads, q_out, stream, true);
+}
+
+int mla_project_output(const uint16_t* o_latent, const uint16_t* w_uv, int tokens, int heads,
+                       uint16_t* o_out, void* stream) {
+  return proj_call(o_latent, nullptr, w_uv, tokens, heads, o_out, stream, false);
+}
+
 int pmla_device_error(void) {
   int dev;
   DeviceInfo* info;

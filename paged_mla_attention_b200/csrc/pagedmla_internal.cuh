@@ -71,6 +71,15 @@ struct AppendParams {
   int batch, s_new, h_kv, max_pages, num_pages;
 };
 
+struct ProjParams {
+  const uint16_t* a;            // absorb: q^C [T][H][128]; project: o^lat [T][H][512]
+  const uint16_t* rope;         // absorb: q^R [T][H][64] (copied to columns 512..575)
+  const uint16_t* w;            // W^UK or W^UV [H][128][512]
+  uint16_t* out;                // absorb: q [T][H][576]; project: o [T][H][128]
+  int* err;                     // device error word
+  int tokens, heads;
+};
+
 // Workspace layout of one decode call: split partials o (chunk-major fp32),
 // their lse, and the per-(sequence, KV head, row group) completion counters the
 // merge kernel waits on.  Returns the total size.
@@ -88,6 +97,7 @@ cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, con
                           const CUtensorMap& tmap_v, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
+cudaError_t launch_proj(const ProjParams& p, bool absorb, cudaStream_t stream);
 size_t decode_smem_bytes();
 
 // Records the message pmla_last_error() returns on this host thread.

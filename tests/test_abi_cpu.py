@@ -109,3 +109,32 @@ def test_append_with_nothing_to_write_is_a_no_op(lib):
     f.restype = I
     assert f(None, None, None, 0, 1, 1, 576, None, 8, 2, None, None) == 0   # empty batch
     assert f(None, None, None, 4, 0, 1, 576, None, 8, 2, None, None) == 0   # no new tokens
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(tokens=-1), -1), (dict(heads=0), -1), (dict(heads=70000), -1),
+    (dict(a=None), -1), (dict(w=None), -1), (dict(out=None), -1), (dict(rope=None), -1),
+    (dict(a=0x1008), -3), (dict(w=0x2004), -3), (dict(rope=0x3002), -3),
+    (dict(out=0x4010), -3),       # outputs need 32-byte alignment (256-bit stores)
+])
+def test_absorb_query_rejects_bad_arguments(lib, kw, code):
+    args = dict(a=0x1000, rope=0x3000, w=0x2000, tokens=4, heads=16, out=0x4000)
+    args.update(kw)
+    P, I = ctypes.c_void_p, ctypes.c_int
+    f = lib.mla_absorb_query
+    f.argtypes = [P, P, P, I, I, P, P]
+    f.restype = I
+    assert f(args["a"], args["rope"], args["w"], args["tokens"], args["heads"], args["out"], None) == code
+
+
+def test_project_output_rejects_bad_arguments(lib):
+    P, I = ctypes.c_void_p, ctypes.c_int
+    f = lib.mla_project_output
+    f.argtypes = [P, P, I, I, P, P]
+    f.restype = I
+    assert f(0x1000, 0x2000, -1, 16, 0x4000, None) == -1
+    assert f(0x1000, 0x2000, 4, 0, 0x4000, None) == -1
+    assert f(None, 0x2000, 4, 16, 0x4000, None) == -1
+    assert f(0x1000, 0x2000, 4, 16, 0x4008, None) == -3
+    assert f(0x1000, 0x2008, 4, 16, 0x4000, None) == -3
+    assert f(None, None, 0, 16, None, None) == 0   # no tokens: nothing to do
