@@ -513,8 +513,9 @@ def bench_append(args):
 def bench_proj(args):
     """The absorbed projections (mla_absorb_query before the decode, mla_project_output
     after it), timed with CUDA events per launch at three token counts with 128 heads.
-    Bytes: activations in and out plus each head's 128 x 512 bf16 weight matrix (read
-    once per 128-token tile); FLOPs 2 x 128 x 512 per (token, head)."""
+    Algorithmic bytes: activations in and out plus each head's 128 x 512 bf16 weight
+    matrix once (the kernels re-read it per 128-token tile, mostly from L2); FLOPs
+    2 x 128 x 512 per (token, head)."""
     import torch
     import paged_mla_attention_b200 as pm
     peaks, _ = load_peaks()
@@ -530,8 +531,7 @@ def bench_proj(args):
         w_uv = (torch.randn((H, 128, 512), device=dev) / 22.6).to(torch.bfloat16)
         q = torch.empty((T, H, 576), dtype=torch.bfloat16, device=dev)
         o = torch.empty((T, H, 128), dtype=torch.bfloat16, device=dev)
-        tiles = (T + 127) // 128
-        wbytes = H * 128 * 512 * 2 * tiles
+        wbytes = H * 128 * 512 * 2
         for name, fn, nbytes in (
                 ("absorb_query", lambda: pm.absorb_query(qn, qr, w_uk, out=q), T * H * (192 + 576) * 2 + wbytes),
                 ("project_output", lambda: pm.project_output(ol, w_uv, out=o), T * H * (512 + 128) * 2 + wbytes)):

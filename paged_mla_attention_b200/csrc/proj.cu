@@ -11,8 +11,10 @@
 //   absorb:   C[t][n] = sum_k q^C[t][k] W^UK[k][n]   M = tokens, N = 512, K = 128
 //             (B = W^UK_h as stored: N contiguous, i.e. MN-major)
 //   unabsorb: C[t][n] = sum_k o^lat[t][k] W^UV[n][k] M = tokens, N = 128, K = 512
-//             (B = W^UV_h as stored: K contiguous, i.e. K-major; K in two halves
-//              so that the operands fit shared memory)
+//             (B = W^UV_h as stored: K contiguous, i.e. K-major; K in four
+//              quarters so that the operands fit shared memory)
+// Operands move with cp.async (16-byte asynchronous copies, many in flight per
+// thread): the kernels are bound by reading each head's 128 KB weight matrix.
 #include "pagedmla_internal.cuh"
 #include "ptx.cuh"
 
@@ -23,46 +25,77 @@ namespace {
 constexpr int kProjThreads = 128;
 constexpr uint32_t kChunk = 16384;  // 128 rows x 128 bytes, one 64-column SW128 chunk
 
-// Row `r` (bytes `src`, `kchunks` x 128 bytes) into chunk-major SW128 K-major layout.
-__device__ __forceinline__ void stage_row(uint8_t* base, const uint8_t* src, int r, int kchunks) {
-  for (int c = 0; c < kchunks; ++c) {
-    const uint4* s = reinterpret_cast<const uint4*>(src + c * 128);
-    uint8_t* d = base + c * kChunk + r * 128;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4*>(d + ((u ^ (r & 7)) << 4)) = __ldg(s + u);
+// 16-byte asynchronous global -> shared copy (L2 only); `src_bytes` 0 fills zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
+}
+
+// Copies 128 rows x `kChunks` 64-column chunks into chunk-major SW128 tiles at
+// `dst` (1024-byte aligned): row r's 16-byte unit u of chunk c lands at
+// c * kChunk + r * 128 + ((u ^ (r & 7)) << 4).  Row r starts at `src` + r * `row_stride`
+// elements (plus `col0`); rows with r >= `rows_valid` are zero-filled.  Eight
+// consecutive threads cover one 128-byte chunk row, so each warp reads whole rows.
+template <int kChunks>
+__device__ __forceinline__ void stage_tile(uint32_t dst, const uint16_t* src, size_t row_stride, int col0,
+                                           int rows_valid, int tid) {
+#pragma unroll 4
+  for (int i = tid; i < 128 * kChunks * 8; i += kProjThreads) {
+    const int u = i & 7, c = (i >> 3) % kChunks, r = (i >> 3) / kChunks;
+    const bool ok = r < rows_valid;
+    const uint16_t* g = ok ? src + (size_t)r * row_stride + col0 + c * 64 + u * 8 : src;
+    cp_async16(dst + c * kChunk + r * 128 + ((u ^ (r & 7)) << 4), g, ok ? 16u : 0u);
   }
 }
 
-__device__ __forceinline__ void zero_row(uint8_t* base, int r, int kchunks) {
-  for (int c = 0; c < kchunks; ++c)
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-      *reinterpret_cast<uint4*>(base + c * kChunk + r * 128 + (u << 4)) = make_uint4(0, 0, 0, 0);
-}
-
+// absorb:  K = 128 in one phase; A (2 chunks) + B (8 N-chunks, MN-major) = 160 KB,
+//          copied as two groups (A and N 0..255, then N 256..511) so the first
+//          N half's MMAs start while the second half lands.
+// project: K = 512 in four phases of 128 (A 2 chunks + B 2 chunks = 64 KB each)
+//          through three buffers; phase 3 reuses buffer 0 once phase 0's MMAs
+//          have completed.
 template <bool kAbsorb>
 __global__ void __launch_bounds__(kProjThreads, 1) proj_kernel(const ProjParams P) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ uint64_t done_bar;
+  __shared__ uint64_t mma_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   constexpr int N = kAbsorb ? 512 : 128;
   constexpr int K = kAbsorb ? 128 : 512;
-  constexpr int kKHalf = kAbsorb ? K : K / 2;  // K staged per phase
-  constexpr int kPhases = K / kKHalf;
-  constexpr int kAChunks = kKHalf / 64;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int t0 = blockIdx.x * 128, h = blockIdx.y;
   const int t = t0 + tid;
   const bool valid = t < P.tokens;
+  const int rows_valid = min(128, P.tokens - t0);
   // the 128-byte swizzle needs 1024-byte aligned tiles: align the dynamic base
   // (one spare KB is part of the allocation)
   const uint32_t raw = smem_u32(smem);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
-  uint8_t* sa = smem + (sbase - raw);                    // A: kAChunks chunks
-  uint8_t* sb = sa + kAChunks * kChunk;                  // B
+  const uint16_t* a = P.a + ((size_t)t0 * P.heads + h) * K;   // token rows of this head
+  const size_t a_stride = (size_t)P.heads * K;
+  const uint16_t* w = P.w + (size_t)h * 128 * 512;             // [128][512]
+
+  if (kAbsorb) {
+    stage_tile<2>(sbase, a, a_stride, 0, rows_valid, tid);                  // A: q^C, K 0..127
+    stage_tile<4>(sbase + 2 * kChunk, w, 512, 0, 128, tid);                 // B: N 0..255
+    cp_async_commit();
+    stage_tile<4>(sbase + 6 * kChunk, w, 512, 256, 128, tid);               // B: N 256..511
+    cp_async_commit();
+  } else {
+#pragma unroll
+    for (int ph = 0; ph < 3; ++ph) {
+      stage_tile<2>(sbase + ph * 4 * kChunk, a, a_stride, ph * 128, rows_valid, tid);
+      stage_tile<2>(sbase + (ph * 4 + 2) * kChunk, w, 512, ph * 128, 128, tid);
+      cp_async_commit();
+    }
+  }
   if (tid == 0) {
-    mbar_init(smem_u32(&done_bar), 1);
+    mbar_init(smem_u32(&mma_bar), 1);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -74,63 +107,72 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_kernel(const ProjParams 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
-  const uint32_t idesc = make_idesc_bf16(128, kAbsorb ? 256 : 128, 0, kAbsorb ? 1 : 0);
+  bool ok = true;
 
-  for (int ph = 0; ph < kPhases; ++ph) {
-    // ---- stage A rows (token t) and B rows (row tid of the head's matrix)
-    if (valid) {
-      const uint8_t* arow =
-          reinterpret_cast<const uint8_t*>(P.a + ((size_t)t * P.heads + h) * K + ph * kKHalf);
-      stage_row(sa, arow, tid, kAChunks);
-    } else {
-      zero_row(sa, tid, kAChunks);
-    }
-    const uint16_t* w = P.w + (size_t)h * 128 * 512;
-    if (kAbsorb) {
-      // W^UK_h row k = tid: 512 N values -> MN-major chunks (64 N columns each)
-      stage_row(sb, reinterpret_cast<const uint8_t*>(w + (size_t)tid * 512), tid, 8);
-    } else {
-      // W^UV_h row n = tid, K half ph: 256 K values -> K-major chunks
-      stage_row(sb, reinterpret_cast<const uint8_t*>(w + (size_t)tid * 512 + ph * kKHalf), tid,
-                kKHalf / 64);
-    }
-    fence_proxy_async_cta();  // generic shared-memory writes -> read by the MMA (async proxy)
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      const uint64_t a0 = make_smem_desc(sbase, 16, 1024, 2);
-      if (kAbsorb) {
-        const uint64_t b0 = make_smem_desc(sbase + kAChunks * kChunk, kChunk, 1024, 2);
+  if (kAbsorb) {
+    const uint32_t idesc = make_idesc_bf16(128, 256, 0, 1);
+    const uint64_t a0 = make_smem_desc(sbase, 16, 1024, 2);
+    const uint64_t b0 = make_smem_desc(sbase + 2 * kChunk, kChunk, 1024, 2);
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+      if (nh == 0) cp_async_wait<1>(); else cp_async_wait<0>();
+      fence_proxy_async_cta();  // cp.async writes (generic proxy) -> read by the MMA
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < K / 16; ++ks) {
           const uint64_t ad = a0 + (uint64_t)(((ks >> 2) * kChunk + (ks & 3) * 32) >> 4);
-#pragma unroll
-          for (int nh = 0; nh < 2; ++nh) {
-            const uint64_t bd = b0 + (uint64_t)((nh * 4 * kChunk + ks * 2048) >> 4);
-            mma_ss(tmem + 256u * nh, ad, bd, idesc, ks > 0);
-          }
+          const uint64_t bd = b0 + (uint64_t)((nh * 4 * kChunk + ks * 2048) >> 4);
+          mma_ss(tmem + 256u * nh, ad, bd, idesc, ks > 0);
         }
-      } else {
-        const uint64_t b0 = make_smem_desc(sbase + kAChunks * kChunk, 16, 1024, 2);
+        if (nh == 1) tc_commit(smem_u32(&mma_bar));
+      }
+    }
+    ok = mbar_wait(smem_u32(&mma_bar), 0u, &abort_flag, P.err, kErrWaitBase + 40);
+  } else {
+    const uint32_t idesc = make_idesc_bf16(128, 128, 0, 0);
 #pragma unroll
-        for (int ks = 0; ks < kKHalf / 16; ++ks) {
+    for (int ph = 0; ph < 4; ++ph) {
+      if (ph == 0) cp_async_wait<2>();
+      else if (ph == 3) cp_async_wait<0>();
+      else cp_async_wait<1>();
+      fence_proxy_async_cta();
+      __syncthreads();
+      const uint32_t buf = sbase + (ph % 3) * 4 * kChunk;
+      if (tid == 0) {
+        tc_fence_after();
+        const uint64_t a0 = make_smem_desc(buf, 16, 1024, 2);
+        const uint64_t b0 = make_smem_desc(buf + 2 * kChunk, 16, 1024, 2);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
           const uint32_t off = ((ks >> 2) * kChunk + (ks & 3) * 32) >> 4;
           mma_ss(tmem, a0 + off, b0 + off, idesc, (ph > 0) || (ks > 0));
         }
+        if (ph == 0 || ph == 3) tc_commit(smem_u32(&mma_bar));
       }
-      tc_commit(smem_u32(&done_bar));
+      if (ph == 1) {
+        // buffer 0 is free once phase 0's MMAs have read it: load phase 3 there
+        ok = __syncthreads_and(mbar_wait(smem_u32(&mma_bar), 0u, &abort_flag, P.err, kErrWaitBase + 40));
+        if (!ok) {
+          cp_async_commit();
+          break;
+        }
+        stage_tile<2>(sbase, a, a_stride, 3 * 128, rows_valid, tid);
+        stage_tile<2>(sbase + 2 * kChunk, w, 512, 3 * 128, 128, tid);
+        cp_async_commit();
+      }
     }
-    // every thread waits for the MMAs (they read this phase's shared memory)
-    const bool ok = mbar_wait(smem_u32(&done_bar), (uint32_t)(ph & 1), &abort_flag, P.err,
-                              kErrWaitBase + 40);
-    if (!__syncthreads_and(ok)) break;
-    tc_fence_after();
+    if (ok) ok = mbar_wait(smem_u32(&mma_bar), 1u, &abort_flag, P.err, kErrWaitBase + 40);
   }
+  cp_async_wait<0>();
+  ok = __syncthreads_and(ok);
+  tc_fence_after();
 
   // ---- epilogue: row tid of the accumulator -> bf16 output row
-  if (!abort_flag) {
+  if (ok) {
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    uint16_t* out = kAbsorb ? P.out + ((size_t)t * P.heads + h) * kD : P.out + ((size_t)t * P.heads + h) * 128;
+    uint16_t* out = P.out + ((size_t)t * P.heads + h) * (kAbsorb ? kD : 128);
 #pragma unroll 1
     for (int j = 0; j < N / 64; ++j) {
       uint32_t v0[32], v1[32];
@@ -166,7 +208,7 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_kernel(const ProjParams 
 }  // namespace
 
 size_t proj_smem_bytes(bool absorb) {
-  return absorb ? (2 + 8) * (size_t)kChunk + 1024 : (4 + 4) * (size_t)kChunk + 1024;
+  return absorb ? (2 + 8) * (size_t)kChunk + 1024 : 3 * 4 * (size_t)kChunk + 1024;
 }
 
 cudaError_t launch_proj(const ProjParams& p, bool absorb, cudaStream_t stream) {
