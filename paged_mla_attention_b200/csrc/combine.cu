@@ -22,9 +22,12 @@
 // resident.  Each finished split piece adds 2 to a counter per (sequence, KV
 // head, row group) -- once after its lse, once after its o rows, each behind
 // a device-scope fence -- and a block merges only after the counter reaches
-// 2 x pieces (a bounded wait that records an error if it runs out).  Blocks
-// end by waiting for the whole decode grid, so work queued after this kernel
-// still sees the decode kernel complete.
+// 2 x pieces (a bounded wait that records an error if it runs out).  The last
+// block of the grid ends by waiting for the whole decode grid, so this grid
+// cannot complete before the decode grid has, and work queued after it sees
+// the decode kernel complete.  Every other block exits as soon as its rows are
+// written: blocks parked on that wait would hold SM slots that blocks still to
+// be dispatched need.
 #include "pagedmla_internal.cuh"
 #include "ptx.cuh"
 
@@ -59,8 +62,10 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombinePar
   const int quarter = blockIdx.x % kQuarters;
   const int s0 = P.num_splits[b];
   const int n = P.num_splits[b + 1] - s0;
+  const bool last_block =
+      blockIdx.x == gridDim.x - 1 && blockIdx.y == gridDim.y - 1 && blockIdx.z == gridDim.z - 1;
   if (n == 1) {  // written by the decode kernel directly
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (last_block) asm volatile("griddepcontrol.wait;" ::: "memory");
     return;
   }
   const int rr = r0 + lane;
@@ -85,7 +90,10 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombinePar
       ready = ok;
     }
     __syncthreads();
-    if (!ready) return;
+    if (!ready) {
+      if (last_block) asm volatile("griddepcontrol.wait;" ::: "memory");
+      return;
+    }
   }
 
   // all lse_k of the block's rows in one round trip (warp w loads pieces w, w+8,
@@ -188,7 +196,7 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombinePar
     const int qi = rr / P.hpk, head = g * P.hpk + rr % P.hpk;
     P.lse[((size_t)b * P.h_q + head) * P.s_q + qi] = row_lse[lane];
   }
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (last_block) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace

@@ -137,8 +137,14 @@ struct Ring {
 };
 
 // Iterates the pieces of a scheduler part: calls f(b, p0, p1, ordinal).
+// Pieces of a part run in sequence order on odd parts and in reverse on even
+// parts.  A sequence cut between parts c and c + 1 then has both of its pieces
+// processed first when c is even (its merge can run while the decode is still
+// going); when c is odd both come last.  In plain order every cut sequence would
+// wait for the end of a part.
 struct PartIter {
   int b0, pg0, b1, pg1, ord0;
+  bool rev;
   __device__ PartIter(const DecodeParams& P, int part) {
     const int32_t* m = P.meta + (size_t)part * kMetaInts;
     b0 = max(m[0], 0);
@@ -146,6 +152,7 @@ struct PartIter {
     b1 = min(m[2], P.batch);
     pg1 = m[3];
     ord0 = max(m[4], 0);
+    rev = (part & 1) == 0;
   }
 };
 
@@ -158,7 +165,9 @@ __device__ __forceinline__ int seq_pages(const DecodeParams& P, int b) {
 
 template <class F>
 __device__ __forceinline__ void for_each_piece(const DecodeParams& P, const PartIter& it, F&& f) {
-  for (int b = it.b0; b <= it.b1 && b < P.batch; ++b) {
+  const int last = min(it.b1, P.batch - 1);
+  for (int k = 0; k <= last - it.b0; ++k) {
+    const int b = it.rev ? last - k : it.b0 + k;
     const int n = seq_pages(P, b);
     const int p0 = (b == it.b0) ? min(it.pg0, n) : 0;
     const int p1 = (b == it.b1) ? min(max(it.pg1, 0), n) : n;
