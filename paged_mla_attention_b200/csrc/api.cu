@@ -423,7 +423,34 @@ static int proj_call(const uint16_t* a, const uint16_t* rope, const uint16_t* w,
   p.err = info->err_ptr;
   p.tokens = tokens;
   p.heads = heads;
-  cudaError_t e = pmla::launch_proj(p, absorb, static_cast<cudaStream_t>(stream));
+  auto encode = get_encode();
+  if (!encode) return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  // activations [tokens][heads][K] as dims {K, heads, tokens}: a box of 64 columns x
+  // 1 head x 128 tokens is one 128-row SW128 chunk of a head's token tile
+  const cuuint64_t K = absorb ? 128 : 512;
+  CUtensorMap tmap_a, tmap_w;
+  {
+    cuuint64_t dim[3] = {K, (cuuint64_t)heads, (cuuint64_t)tokens};
+    cuuint64_t stride[2] = {K * 2, (cuuint64_t)heads * K * 2};
+    cuuint32_t box[3] = {64, 1, 128};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult cr = encode(&tmap_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(a), dim, stride,
+                         box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled (activations) failed (%d)", (int)cr);
+  }
+  // weights [heads][128][512] as dims {512, heads*128}: a box of 64 columns x 128 rows
+  {
+    cuuint64_t dim[2] = {512, (cuuint64_t)heads * 128};
+    cuuint64_t stride[1] = {1024};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t es[2] = {1, 1};
+    CUresult cr = encode(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(w), dim, stride,
+                         box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled (weights) failed (%d)", (int)cr);
+  }
+  cudaError_t e = pmla::launch_proj(p, absorb, tmap_a, tmap_w, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e, "projection kernel launch");
   return PMLA_OK;
 }

@@ -97,7 +97,8 @@ cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, con
                           const CUtensorMap& tmap_v, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
-cudaError_t launch_proj(const ProjParams& p, bool absorb, cudaStream_t stream);
+cudaError_t launch_proj(const ProjParams& p, bool absorb, const CUtensorMap& tmap_a, const CUtensorMap& tmap_w,
+                        cudaStream_t stream);
 size_t decode_smem_bytes();
 
 // Records the message pmla_last_error() returns on this host thread.

@@ -13,8 +13,9 @@
 //   unabsorb: C[t][n] = sum_k o^lat[t][k] W^UV[n][k] M = tokens, N = 128, K = 512
 //             (B = W^UV_h as stored: K contiguous, i.e. K-major; K in four
 //              quarters so that the operands fit shared memory)
-// Operands move with cp.async (16-byte asynchronous copies, many in flight per
-// thread): the kernels are bound by reading each head's 128 KB weight matrix.
+// Operands move by TMA (one thread issues every tile of the CTA, so a whole
+// head's weight matrix is in flight at once): the kernels are bound by reading
+// each head's 128 KB weight matrix.  Tokens past the end read as zeros.
 #include "pagedmla_internal.cuh"
 #include "ptx.cuh"
 
@@ -25,79 +26,43 @@ namespace {
 constexpr int kProjThreads = 128;
 constexpr uint32_t kChunk = 16384;  // 128 rows x 128 bytes, one 64-column SW128 chunk
 
-// 16-byte asynchronous global -> shared copy (L2 only); `src_bytes` 0 fills zeros.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int kPending>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
-}
-
-// Copies 128 rows x `kChunks` 64-column chunks into chunk-major SW128 tiles at
-// `dst` (1024-byte aligned): row r's 16-byte unit u of chunk c lands at
-// c * kChunk + r * 128 + ((u ^ (r & 7)) << 4).  Row r starts at `src` + r * `row_stride`
-// elements (plus `col0`); rows with r >= `rows_valid` are zero-filled.  Eight
-// consecutive threads cover one 128-byte chunk row, so each warp reads whole rows.
-template <int kChunks>
-__device__ __forceinline__ void stage_tile(uint32_t dst, const uint16_t* src, size_t row_stride, int col0,
-                                           int rows_valid, int tid) {
-#pragma unroll 4
-  for (int i = tid; i < 128 * kChunks * 8; i += kProjThreads) {
-    const int u = i & 7, c = (i >> 3) % kChunks, r = (i >> 3) / kChunks;
-    const bool ok = r < rows_valid;
-    const uint16_t* g = ok ? src + (size_t)r * row_stride + col0 + c * 64 + u * 8 : src;
-    cp_async16(dst + c * kChunk + r * 128 + ((u ^ (r & 7)) << 4), g, ok ? 16u : 0u);
-  }
-}
-
-// absorb:  K = 128 in one phase; A (2 chunks) + B (8 N-chunks, MN-major) = 160 KB,
-//          copied as two groups (A and N 0..255, then N 256..511) so the first
-//          N half's MMAs start while the second half lands.
+// Chunks are filled by TMA boxes of 64 columns x 128 rows (128-byte swizzle):
+//   a map:  [T][H][K] as dims {K, H, T}, box {64, 1, 128}: 128 tokens of head h
+//   w map:  [H*128][512] as dims {512, H*128}, box {64, 128}: 128 rows of head h
+// absorb:  K = 128 in one phase; A (2 chunks) + B (8 N-chunks, MN-major) = 160 KB
+//          behind two barriers (A and N 0..255, then N 256..511) so the first N
+//          half's MMAs start while the second half lands.
 // project: K = 512 in four phases of 128 (A 2 chunks + B 2 chunks = 64 KB each)
 //          through three buffers; phase 3 reuses buffer 0 once phase 0's MMAs
 //          have completed.
+// Thread 0 issues the copies and the MMAs; all threads run the epilogue.
 template <bool kAbsorb>
-__global__ void __launch_bounds__(kProjThreads, 1) proj_kernel(const ProjParams P) {
+__global__ void __launch_bounds__(kProjThreads, 1)
+proj_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
+            const ProjParams P) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ uint64_t mma_bar;
+  __shared__ uint64_t full_bar[3];
+  __shared__ uint64_t mma_bar[2];
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   constexpr int N = kAbsorb ? 512 : 128;
-  constexpr int K = kAbsorb ? 128 : 512;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int t0 = blockIdx.x * 128, h = blockIdx.y;
   const int t = t0 + tid;
   const bool valid = t < P.tokens;
-  const int rows_valid = min(128, P.tokens - t0);
   // the 128-byte swizzle needs 1024-byte aligned tiles: align the dynamic base
   // (one spare KB is part of the allocation)
   const uint32_t raw = smem_u32(smem);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
-  const uint16_t* a = P.a + ((size_t)t0 * P.heads + h) * K;   // token rows of this head
-  const size_t a_stride = (size_t)P.heads * K;
-  const uint16_t* w = P.w + (size_t)h * 128 * 512;             // [128][512]
+  const int wrow = h * 128;  // first row of this head's weight matrix
 
-  if (kAbsorb) {
-    stage_tile<2>(sbase, a, a_stride, 0, rows_valid, tid);                  // A: q^C, K 0..127
-    stage_tile<4>(sbase + 2 * kChunk, w, 512, 0, 128, tid);                 // B: N 0..255
-    cp_async_commit();
-    stage_tile<4>(sbase + 6 * kChunk, w, 512, 256, 128, tid);               // B: N 256..511
-    cp_async_commit();
-  } else {
-#pragma unroll
-    for (int ph = 0; ph < 3; ++ph) {
-      stage_tile<2>(sbase + ph * 4 * kChunk, a, a_stride, ph * 128, rows_valid, tid);
-      stage_tile<2>(sbase + (ph * 4 + 2) * kChunk, w, 512, ph * 128, 128, tid);
-      cp_async_commit();
-    }
-  }
   if (tid == 0) {
-    mbar_init(smem_u32(&mma_bar), 1);
+    for (int i = 0; i < 3; ++i) mbar_init(smem_u32(&full_bar[i]), 1);
+    for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&mma_bar[i]), 1);
     abort_flag = 0;
     fence_mbar_init();
+    tma_prefetch_desc(&tmap_a);
+    tma_prefetch_desc(&tmap_w);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(&tmem_base), N);
@@ -107,66 +72,83 @@ __global__ void __launch_bounds__(kProjThreads, 1) proj_kernel(const ProjParams 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
-  bool ok = true;
 
-  if (kAbsorb) {
-    const uint32_t idesc = make_idesc_bf16(128, 256, 0, 1);
-    const uint64_t a0 = make_smem_desc(sbase, 16, 1024, 2);
-    const uint64_t b0 = make_smem_desc(sbase + 2 * kChunk, kChunk, 1024, 2);
-#pragma unroll
-    for (int nh = 0; nh < 2; ++nh) {
-      if (nh == 0) cp_async_wait<1>(); else cp_async_wait<0>();
-      fence_proxy_async_cta();  // cp.async writes (generic proxy) -> read by the MMA
-      __syncthreads();
-      if (tid == 0) {
+  if (tid == 0) {
+    const uint64_t pol_a = policy_evict_first();
+    const uint64_t pol_w = policy_evict_last();  // re-read by the head's other token tiles
+    bool ok = true;
+    uint32_t issued = 0;  // bit i: full_bar[i] has a phase in flight
+    uint32_t issued_par = 0;  // bit i: the parity of that phase
+    if (kAbsorb) {
+      const uint32_t f0 = smem_u32(&full_bar[0]), f1 = smem_u32(&full_bar[1]);
+      mbar_arrive_expect_tx(f0, 6 * kChunk);
+      for (int c = 0; c < 2; ++c) tma_load_3d(sbase + c * kChunk, &tmap_a, f0, c * 64, h, t0, pol_a);
+      for (int c = 0; c < 4; ++c) tma_load_2d(sbase + (2 + c) * kChunk, &tmap_w, f0, c * 64, wrow, pol_w);
+      mbar_arrive_expect_tx(f1, 4 * kChunk);
+      for (int c = 4; c < 8; ++c) tma_load_2d(sbase + (2 + c) * kChunk, &tmap_w, f1, c * 64, wrow, pol_w);
+      issued = 3u;
+      const uint32_t idesc = make_idesc_bf16(128, 256, 0, 1);
+      const uint64_t a0 = make_smem_desc(sbase, 16, 1024, 2);
+      const uint64_t b0 = make_smem_desc(sbase + 2 * kChunk, kChunk, 1024, 2);
+      for (int nh = 0; nh < 2 && ok; ++nh) {
+        ok = mbar_wait(nh ? f1 : f0, 0u, &abort_flag, P.err, kErrWaitBase + 40);
+        if (!ok) break;
+        issued &= ~(1u << nh);
         tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < K / 16; ++ks) {
+        for (int ks = 0; ks < 8; ++ks) {
           const uint64_t ad = a0 + (uint64_t)(((ks >> 2) * kChunk + (ks & 3) * 32) >> 4);
           const uint64_t bd = b0 + (uint64_t)((nh * 4 * kChunk + ks * 2048) >> 4);
           mma_ss(tmem + 256u * nh, ad, bd, idesc, ks > 0);
         }
-        if (nh == 1) tc_commit(smem_u32(&mma_bar));
       }
-    }
-    ok = mbar_wait(smem_u32(&mma_bar), 0u, &abort_flag, P.err, kErrWaitBase + 40);
-  } else {
-    const uint32_t idesc = make_idesc_bf16(128, 128, 0, 0);
-#pragma unroll
-    for (int ph = 0; ph < 4; ++ph) {
-      if (ph == 0) cp_async_wait<2>();
-      else if (ph == 3) cp_async_wait<0>();
-      else cp_async_wait<1>();
-      fence_proxy_async_cta();
-      __syncthreads();
-      const uint32_t buf = sbase + (ph % 3) * 4 * kChunk;
-      if (tid == 0) {
+      if (ok) tc_commit(smem_u32(&mma_bar[1]));
+    } else {
+      auto load_phase = [&](int ph, int buf) {
+        const uint32_t f = smem_u32(&full_bar[buf]);
+        const uint32_t dst = sbase + buf * 4 * kChunk;
+        mbar_arrive_expect_tx(f, 4 * kChunk);
+        issued_par = (issued_par & ~(1u << buf)) | ((uint32_t)(ph / 3) << buf);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(dst + c * kChunk, &tmap_a, f, ph * 128 + c * 64, h, t0, pol_a);
+          tma_load_2d(dst + (2 + c) * kChunk, &tmap_w, f, ph * 128 + c * 64, wrow, pol_w);
+        }
+        issued |= 1u << buf;
+      };
+      for (int ph = 0; ph < 3; ++ph) load_phase(ph, ph);
+      const uint32_t idesc = make_idesc_bf16(128, 128, 0, 0);
+      for (int ph = 0; ph < 4 && ok; ++ph) {
+        const int buf = ph % 3;
+        ok = mbar_wait(smem_u32(&full_bar[buf]), (uint32_t)(ph / 3), &abort_flag, P.err, kErrWaitBase + 40);
+        if (!ok) break;
+        issued &= ~(1u << buf);
         tc_fence_after();
-        const uint64_t a0 = make_smem_desc(buf, 16, 1024, 2);
-        const uint64_t b0 = make_smem_desc(buf + 2 * kChunk, 16, 1024, 2);
+        const uint32_t base = sbase + buf * 4 * kChunk;
+        const uint64_t a0 = make_smem_desc(base, 16, 1024, 2);
+        const uint64_t b0 = make_smem_desc(base + 2 * kChunk, 16, 1024, 2);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t off = ((ks >> 2) * kChunk + (ks & 3) * 32) >> 4;
           mma_ss(tmem, a0 + off, b0 + off, idesc, (ph > 0) || (ks > 0));
         }
-        if (ph == 0 || ph == 3) tc_commit(smem_u32(&mma_bar));
-      }
-      if (ph == 1) {
-        // buffer 0 is free once phase 0's MMAs have read it: load phase 3 there
-        ok = __syncthreads_and(mbar_wait(smem_u32(&mma_bar), 0u, &abort_flag, P.err, kErrWaitBase + 40));
-        if (!ok) {
-          cp_async_commit();
-          break;
+        if (ph == 0) {
+          tc_commit(smem_u32(&mma_bar[0]));
+        } else if (ph == 1) {
+          // buffer 0 is free once phase 0's MMAs have read it: load phase 3 there
+          ok = mbar_wait(smem_u32(&mma_bar[0]), 0u, &abort_flag, P.err, kErrWaitBase + 40);
+          if (ok) load_phase(3, 0);
         }
-        stage_tile<2>(sbase, a, a_stride, 3 * 128, rows_valid, tid);
-        stage_tile<2>(sbase + 2 * kChunk, w, 512, 3 * 128, 128, tid);
-        cp_async_commit();
       }
+      if (ok) tc_commit(smem_u32(&mma_bar[1]));
     }
-    if (ok) ok = mbar_wait(smem_u32(&mma_bar), 1u, &abort_flag, P.err, kErrWaitBase + 40);
+    if (!ok) {  // no copy may still be writing this CTA's shared memory when it exits
+      abort_flag = 1;
+      for (int i = 0; i < 3; ++i)
+        if (issued & (1u << i)) mbar_wait_drain(smem_u32(&full_bar[i]), (issued_par >> i) & 1u);
+    }
   }
-  cp_async_wait<0>();
-  ok = __syncthreads_and(ok);
+  // every thread waits for the accumulator
+  const bool ok = __syncthreads_and(mbar_wait(smem_u32(&mma_bar[1]), 0u, &abort_flag, P.err, kErrWaitBase + 40));
   tc_fence_after();
 
   // ---- epilogue: row tid of the accumulator -> bf16 output row
@@ -211,7 +193,8 @@ size_t proj_smem_bytes(bool absorb) {
   return absorb ? (2 + 8) * (size_t)kChunk + 1024 : 3 * 4 * (size_t)kChunk + 1024;
 }
 
-cudaError_t launch_proj(const ProjParams& p, bool absorb, cudaStream_t stream) {
+cudaError_t launch_proj(const ProjParams& p, bool absorb, const CUtensorMap& tmap_a, const CUtensorMap& tmap_w,
+                        cudaStream_t stream) {
   if (p.tokens == 0) return cudaSuccess;
   const size_t smem = proj_smem_bytes(absorb);
   cudaError_t e = absorb ? cudaFuncSetAttribute(proj_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
@@ -219,9 +202,9 @@ cudaError_t launch_proj(const ProjParams& p, bool absorb, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   dim3 grid((p.tokens + 127) / 128, p.heads);
   if (absorb)
-    proj_kernel<true><<<grid, kProjThreads, smem, stream>>>(p);
+    proj_kernel<true><<<grid, kProjThreads, smem, stream>>>(tmap_a, tmap_w, p);
   else
-    proj_kernel<false><<<grid, kProjThreads, smem, stream>>>(p);
+    proj_kernel<false><<<grid, kProjThreads, smem, stream>>>(tmap_a, tmap_w, p);
   return cudaGetLastError();
 }
 
