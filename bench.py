@@ -385,7 +385,7 @@ def bench_ours(args, rank, world, local_rank):
         "e2e": {"value": round(world * wc["kv_bytes"] / (e2e_ms / 1e3 / e2e_steps) / 1e9, 3), "unit": "GB/s",
                 "steps": e2e_steps, "ms_per_step": round(e2e_ms / e2e_steps, 4),
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
-        "gpu_launches": 3 * K,  # schedule, decode, merge per timed step
+        "gpu_launches": 4 * K,  # schedule, counter clear, decode, merge per timed step
         "clocks": clk.summary(),
     }
     if spot is not None:

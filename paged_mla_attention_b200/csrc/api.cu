@@ -314,7 +314,7 @@ int decode_impl(const uint16_t* q, const uint16_t* kvcache, const int32_t* block
     cudaError_t e = pmla::decode_prepare(dev);
     if (e != cudaSuccess) return fail_cuda(e, "decode kernel attributes");
     // the merge kernel counts completion signals from zero
-    e = cudaMemsetAsync(p.seq_done, 0, wl.done_count * sizeof(int), st);
+    e = pmla::launch_clear_counters(p.seq_done, (int)wl.done_count, st);
     if (e != cudaSuccess) return fail_cuda(e, "clearing the completion counters");
     e = pmla::launch_decode(p, tmap, tmap_q, tmap_v, st);
     if (e != cudaSuccess) return fail_cuda(e, "decode kernel launch");

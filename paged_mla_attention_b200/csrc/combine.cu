@@ -201,6 +201,35 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombinePar
 
 }  // namespace
 
+namespace {
+
+// Zeroes the merge's completion counters.  Launched as a programmatic dependent
+// of whatever precedes it (normally the schedule), it lets its own dependent,
+// the decode kernel, start its setup at once; it zeroes only after the
+// preceding grid has completed (a decode kernel of an earlier call may still be
+// counting), so when this grid completes, so has the one before it.
+__global__ void __launch_bounds__(256) clear_counters_kernel(int* ctr, int n) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) ctr[i] = 0;
+}
+
+}  // namespace
+
+cudaError_t launch_clear_counters(int* ctr, int n, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((n + 255) / 256 < 148 ? (n + 255) / 256 : 148), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, clear_counters_kernel, ctr, n);
+}
+
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
   if (p.batch == 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};

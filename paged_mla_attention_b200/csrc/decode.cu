@@ -284,6 +284,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
   cluster_wait();
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem_base;
+  // launched as a programmatic dependent of the counter clear: the setup above
+  // overlaps the kernels before it; the schedule and the cleared counters are
+  // read only after this wait (the clear's grid completes after the schedule's)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // every CTA of this grid is resident now: the merge kernel, launched as a
   // programmatic dependent, may start on SMs as they free up (it waits for the
   // completion signals of the pieces it merges)
@@ -932,8 +936,17 @@ int decode_max_active_clusters(int device, int* out) {
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, const CUtensorMap& tmap_q,
                           const CUtensorMap& tmap_v, cudaStream_t stream) {
   const int clusters = p.num_parts * p.h_kv * p.n_rg;
-  decode_kernel<<<2 * clusters, kThreads, SMEM_BYTES, stream>>>(tmap_kv, tmap_q, tmap_v, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_kernel, tmap_kv, tmap_q, tmap_v, p);
 }
 
 }  // namespace pmla

@@ -96,6 +96,7 @@ int decode_max_active_clusters(int device, int* out);
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, const CUtensorMap& tmap_q,
                           const CUtensorMap& tmap_v, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
+cudaError_t launch_clear_counters(int* ctr, int n, cudaStream_t stream);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 cudaError_t launch_proj(const ProjParams& p, bool absorb, const CUtensorMap& tmap_a, const CUtensorMap& tmap_w,
                         cudaStream_t stream);

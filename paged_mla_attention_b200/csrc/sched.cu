@@ -82,6 +82,9 @@ __global__ void __launch_bounds__(kSchedThreads) metadata_kernel(const int32_t* 
   __shared__ int cut_seq[kMaxParts];       // sequence of each distinct cut, in order
   __shared__ int sh_ncuts;
 
+  // the kernel queued next may start now (the counter clear, then the decode
+  // kernel's setup); they wait for this grid before reading what it writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const long long F = kPieceCostPages;
   const int t = threadIdx.x;
   const int P = num_parts;
