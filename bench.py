@@ -259,9 +259,10 @@ def bench_ours(args, rank, world, local_rank):
     if err:
         raise RuntimeError(f"device error {err} during warm-up")
 
-    # CUDA graphs: the schedule; the decode call (decode kernel, then the merge
-    # kernel as a programmatic dependent that overlaps the decode tail); and the
-    # decode kernel alone, for the roofline
+    # CUDA graphs: the whole step (schedule, counter clear, decode kernel, merge
+    # kernel: a programmatic launch chain, so each kernel's launch overlaps the
+    # one before); the decode call alone (schedule excluded); and the decode
+    # kernel alone, for the roofline
     g_meta, g_all, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_meta, stream=stream):
         step_meta()
@@ -269,8 +270,13 @@ def bench_ours(args, rank, world, local_rank):
         step_decode("all")
     with torch.cuda.graph(g_dec, stream=stream):
         step_decode("decode")
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=stream):
+        step_meta()
+        step_decode("all")
     for _ in range(3):
-        g_meta.replay()
+        g_meta.replay()  # fills the schedule that g_all and g_dec read
+        g_step.replay()
         g_all.replay()
         g_dec.replay()
     torch.cuda.synchronize(dev)
@@ -278,8 +284,7 @@ def bench_ours(args, rank, world, local_rank):
     K = args.steps
     ev_start = torch.cuda.Event(enable_timing=True)
     ev_end = torch.cuda.Event(enable_timing=True)
-    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -287,14 +292,16 @@ def bench_ours(args, rank, world, local_rank):
     with ClockSampler(local_rank) as clk:
         ev_start.record()
         for k in range(K):
-            g_meta.replay()
-            ev_a[k].record()
-            g_all.replay()
-            ev_b[k].record()
+            g_step.replay()
         ev_end.record()
         torch.cuda.synchronize(dev)
-        # the decode kernel alone, K more launches right after the timed steps
-        # (same stream, same inputs), each bracketed by events
+        # the decode call alone, then the decode kernel alone: K more launches each
+        # right after the timed steps (same stream, same inputs), each bracketed by events
+        ev_a[0].record()
+        for k in range(K):
+            g_all.replay()
+            ev_a[k + 1].record()
+        torch.cuda.synchronize(dev)
         ev_c = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
         ev_c[0].record()
         for k in range(K):
@@ -304,7 +311,7 @@ def bench_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     elapsed_ms = ev_start.elapsed_time(ev_end)
-    call_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]))  # decode + merge
+    call_ms = float(np.mean([ev_a[k].elapsed_time(ev_a[k + 1]) for k in range(K)]))  # clear + decode + merge
     dec_ms = float(np.mean([ev_c[k].elapsed_time(ev_c[k + 1]) for k in range(K)]))  # decode kernel
     err = pm.device_error()
     if err:
@@ -369,7 +376,7 @@ def bench_ours(args, rank, world, local_rank):
         "config": {"workload": workload_desc(w), "global_batch": inp["batch"] * world,
                    "kv_tokens_per_gpu": wc["tokens"], "parallelism": f"replicas x{world} (batch-sharded, no exchange)",
                    "l2": "inputs (302 MB KV) larger than the 126 MB L2; no flush",
-                   "step": "schedule + split-KV decode + merge, replayed from CUDA graphs"},
+                   "step": "schedule + counter clear + split-KV decode + merge, one CUDA graph per step"},
         "us_decode_kernel": round(dec_ms * 1e3, 3),
         "us_per_call": round(call_ms * 1e3, 3),
         "tflops": round(wc["flops"] / dec_s / 1e12, 2),
