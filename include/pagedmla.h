@@ -126,11 +126,19 @@ PMLA_API int mla_get_metadata(const int32_t* cache_seqlens, int batch, int num_h
  *                 mla_get_metadata_sizes; contents need not be initialised;
  *                 must not be shared by calls that may run concurrently.
  * Alignment: q and kvcache 16-byte aligned; o and workspace 32-byte aligned.
+ * batch = 0 returns PMLA_OK once the shape arguments are valid, without looking
+ * at any pointer (empty tensors may be null) and without launching anything.
  * Errors: INVALID_ARG, UNSUPPORTED (d != 576, dv != 512, h_q % h_kv != 0, or
  *         h_q/h_kv neither a divisor of 128 that is >= 8 nor a multiple of 128),
  *         ALIGNMENT, WORKSPACE, CUDA.
  * Device-side waits are bounded; a kernel that gives up records an error that
  * pmla_device_error() returns.
+ * Launches: a counter-clear kernel, the decode kernel and the merge kernel, the
+ * last three as a programmatic launch chain (each may start its setup while the
+ * one before runs, and waits for it before reading its results).  The schedule
+ * kernel of mla_get_metadata lets the next kernel start early the same way;
+ * kernels of the caller that are not launched as programmatic dependents are
+ * ordered as usual.
  */
 PMLA_API int mla_decode_with_kvcache(const uint16_t* q, const uint16_t* kvcache, const int32_t* block_table,
                             const int32_t* cache_seqlens, int batch, int s_q, int h_q, int h_kv,

@@ -212,6 +212,7 @@ int decode_impl(const uint16_t* q, const uint16_t* kvcache, const int32_t* block
     return fail(PMLA_ERR_UNSUPPORTED, "kv cache too large for 32-bit row coordinates");
   if (!std::isfinite(softmax_scale) || softmax_scale < 0.f)
     return fail(PMLA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  if (batch == 0) return PMLA_OK;  // nothing to read or write: buffers may be empty (null)
   if (!q || !kvcache || !block_table || !cache_seqlens || !tile_scheduler_metadata ||
       !num_splits || !o || !lse)
     return fail(PMLA_ERR_INVALID_ARG, "null pointer argument");
@@ -224,7 +225,6 @@ int decode_impl(const uint16_t* q, const uint16_t* kvcache, const int32_t* block
   if (!workspace || workspace_bytes < need || !aligned32(workspace))
     return fail(PMLA_ERR_WORKSPACE, "workspace needs %zu bytes, 32-byte aligned (got %zu)", need,
                 workspace_bytes);
-  if (batch == 0) return PMLA_OK;
 
   int dev;
   DeviceInfo* info;

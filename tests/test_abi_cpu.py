@@ -138,3 +138,10 @@ def test_project_output_rejects_bad_arguments(lib):
     assert f(0x1000, 0x2000, 4, 16, 0x4008, None) == -3
     assert f(0x1000, 0x2008, 4, 16, 0x4000, None) == -3
     assert f(None, None, 0, 16, None, None) == 0   # no tokens: nothing to do
+
+
+def test_decode_with_empty_batch_is_a_no_op(lib):
+    # nothing to read or write: every pointer may be null (empty tensors)
+    assert _decode(lib, batch=0, q=None, kv=None, bt=None, sl=None, meta=None, splits=None, o=None,
+                   lse=None, ws=None, ws_bytes=0) == 0
+    assert _decode(lib, batch=0, d=575) == -2       # shapes are still checked

@@ -208,3 +208,29 @@ def test_full_size_configs_sampled(name):
     sub = subset(inp, seqs, heads)
     ro, rl = oracle.decode_inputs(sub)
     compare(o[seqs][:, :, heads], lse[seqs][:, heads], ro, rl, what=name)
+
+
+def test_empty_batch():
+    import torch
+    import paged_mla_attention_b200 as pm
+    sl = torch.empty((0,), dtype=torch.int32, device="cuda")
+    meta, splits = pm.get_mla_metadata(sl, 128, 1)
+    q = torch.empty((0, 1, 128, W.D_QK), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((1, 64, 1, W.D_QK), dtype=torch.bfloat16, device="cuda")
+    bt = torch.zeros((0, 1), dtype=torch.int32, device="cuda")
+    o, lse = pm.flash_mla_with_kvcache(q, kv, bt, sl, W.D_V, meta, splits)
+    torch.cuda.synchronize()
+    assert pm.device_error() == 0
+    assert tuple(o.shape) == (0, 1, 128, W.D_V) and tuple(lse.shape) == (0, 128, 1)
+    assert splits.cpu().tolist() == [0]
+
+
+def test_all_sequences_empty():
+    # every row sees nothing: o = 0, lse = -inf (no merge work, no NaN)
+    stats, _, splits = _check(_small([0, 0, 0], h_q=64, seed=31), "all empty")
+    assert list(splits) == [0, 0, 0, 0]
+
+
+def test_four_query_tokens_128_heads():
+    # s_q = 4 x h_q = 128: four 128-row groups per KV head, causal
+    _check(_small([3, 64, 200, 1000], s_q=4, h_q=128, causal=True, seed=32), "s_q=4 h_q=128")
