@@ -234,3 +234,27 @@ def test_all_sequences_empty():
 def test_four_query_tokens_128_heads():
     # s_q = 4 x h_q = 128: four 128-row groups per KV head, causal
     _check(_small([3, 64, 200, 1000], s_q=4, h_q=128, causal=True, seed=32), "s_q=4 h_q=128")
+
+
+def test_back_to_back_calls_share_a_workspace():
+    # two decode calls queued on one stream with no host sync in between, on the same
+    # workspace: the second call's counter clear must wait for the first decode
+    # (programmatic launch chain) and both results must match the oracle
+    import torch
+    import paged_mla_attention_b200 as pm
+    a = _small([9000, 100, 3000, 64], h_q=128, seed=41)
+    b = _small([300, 7000, 1, 2500], h_q=128, seed=42)
+    da, db = to_device(a), to_device(b)
+    ws = torch.empty((pm.workspace_bytes(4, 1, 128, 1),), dtype=torch.uint8, device="cuda")
+    outs = []
+    for inp, d in ((a, da), (b, db)):
+        meta, splits = pm.get_mla_metadata(d["cache_seqlens"], 128, 1)
+        outs.append(pm.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"],
+                                              W.D_V, meta, splits, softmax_scale=inp["softmax_scale"],
+                                              workspace=ws))
+    torch.cuda.synchronize()
+    assert pm.device_error() == 0
+    for inp, (o, lse) in zip((a, b), outs):
+        ro, rl = oracle.decode_inputs(inp)
+        compare(o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64), ro, rl,
+                what="back to back")
