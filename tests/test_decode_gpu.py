@@ -258,3 +258,21 @@ def test_back_to_back_calls_share_a_workspace():
         ro, rl = oracle.decode_inputs(inp)
         compare(o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64), ro, rl,
                 what="back to back")
+
+
+@pytest.mark.parametrize("batch", [1500, 5000])
+def test_large_batch_schedule_and_sampled_parity(batch):
+    # more sequences than scheduler threads: each thread owns a chunk of several
+    # sequences; the merge grid spans thousands of sequences
+    rng = np.random.default_rng(batch)
+    lens = rng.integers(0, 400, size=batch)
+    lens[rng.choice(batch, size=batch // 50, replace=False)] = rng.integers(2000, 9000, size=batch // 50)
+    inp = _small(lens.tolist(), h_q=16, seed=batch, extra_pages=2)
+    o, lse, meta, splits = run_gpu(inp)
+    check_schedule(meta, splits, inp["cache_seqlens"], meta.shape[0])
+    assert np.isfinite(o).all()
+    pick = sorted({int(np.argmax(lens)), int(np.argmin(lens)), 0, batch - 1,
+                   *[int(x) for x in rng.choice(batch, size=6, replace=False)]})
+    sub = subset(inp, pick)
+    ro, rl = oracle.decode_inputs(sub)
+    compare(o[pick], lse[pick], ro, rl, what=f"batch {batch}")
