@@ -15,29 +15,34 @@
 // does not fit one SM, so every work unit is a 2-CTA cluster with split roles:
 //
 //   CTA 0 ("S-CTA"): the latent part of Q (512 columns) lives in TMEM as an MMA
-//     A operand (256 columns), its RoPE part (64 columns) in shared memory; S
-//     is double-buffered in the other 2 x 128 TMEM columns.  A TMA warp
-//     streams 16 KB chunk stages through a 13-stage ring: chunk c of two
-//     consecutive pages (rows 0-63 page A, rows 64-127 page B, 64 columns,
-//     128B swizzle), so one MMA covers 128 tokens (N = 128 runs the tensor
-//     core at full rate, N = 64 does not).  One thread issues per page pair
-//     32 TS MMAs (latent, A from TMEM) + 4 SS MMAs (RoPE).  Four softmax warps
-//     (one row per thread) read S, apply the mask, keep the running max/sum in
-//     fp32 with a lazy rescale (the reference max only moves when a pair's max
-//     exceeds it by 2^8), and push P (bf16, swizzled K-major MMA layout) plus
-//     per-row factors into CTA 1's shared memory with st.async, which
-//     completes bytes on CTA 1's barrier: no fence, no extra arrival.
-//     The query tile itself arrives through the same ring (TMA), and the
-//     softmax warps copy its latent chunks into TMEM.
+//     A operand (256 columns of bf16 pairs), its RoPE part (64 columns) in
+//     shared memory; S is double-buffered in the other 2 x 128 TMEM columns.
+//     Two TMA producer threads stream 16 KB chunk stages through an 8-stage
+//     ring: chunk c of two consecutive pages (rows 0-63 page A, rows 64-127
+//     page B, 64 columns, 128B swizzle; one producer per page), so one MMA
+//     covers 128 tokens (N = 128 runs the tensor core at full rate, N = 64
+//     does not).  The query arrives through the same ring; the MMA thread
+//     copies its latent chunks into TMEM (tcgen05.cp) and issues per page pair
+//     32 TS MMAs (latent, A from TMEM) + 4 SS MMAs (RoPE).  Two softmax
+//     warpgroups (one row per thread, one page of the pair each) read S, apply
+//     the mask, exchange row maxima, keep the running max/sum in fp32 with a
+//     lazy rescale (the reference max only moves when a pair's max exceeds it
+//     by 2^8), stage P (bf16, swizzled K-major MMA layout) plus per-row
+//     factors in shared memory, and one thread bulk-copies them into a P slot
+//     of CTA 1, completing bytes on CTA 1's slot barrier.
 //   CTA 1 ("O-CTA"): a TMA warp streams the value part of the same pages in
 //     32 KB half-page stages (mostly L2 hits: CTA 0 just read the page); one
 //     thread issues O += P V as 8 MMAs per page (M=128, N=256, K=16, V
 //     MN-major) into the 512-column accumulator; a relay warp re-arms each
-//     consumed P slot's barrier with its byte count and returns the slot to
-//     CTA 0; four correction warps rescale O rows when CTA 0 moved a row's
-//     reference max, and run the epilogue (O / l -> bf16 o, or fp32 partials)
-//     at the end of each piece.
+//     consumed P slot's barrier and returns the slot to CTA 0; two correction
+//     warpgroups (256 accumulator columns each) sum the bf16 weights they see
+//     into the row sums, rescale O rows when CTA 0 moved a row's reference
+//     max, and run the epilogue (O / l -> bf16 o, or fp32 partials) at the end
+//     of each piece.
 //
+// Launch: a programmatic dependent of the counter-clear kernel (setup overlaps
+// the kernels before it; the schedule is read after griddepcontrol.wait); its
+// own dependent, the merge kernel, may start as soon as every CTA is resident.
 // Every wait is bounded (see ptx.cuh); a timeout records an error code and
 // makes all roles leave their loops, drain their in-flight copies and MMAs,
 // free TMEM and exit.
