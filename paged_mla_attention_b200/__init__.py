@@ -7,6 +7,10 @@ The two calls mirror the FlashMLA usage the DeepSeek pages show (usage steps
     o, lse = flash_mla_with_kvcache(q, kvcache, block_table, cache_seqlens, dv,
                                     tile_scheduler_metadata, num_splits, causal=True)
 
+Around them: ``append_kvcache`` (new tokens into their pages), ``PagePool`` (host
+page allocator), ``absorb_query`` / ``project_output`` (the absorbed W^UK / W^UV
+projections), ``metadata_sizes`` / ``workspace_bytes`` and ``device_error``.
+
 This module only marshals arguments: it checks tensor dtypes/devices, allocates
 the outputs and the split workspace with torch, and passes raw device pointers
 and the current CUDA stream to the C ABI (``include/pagedmla.h``).  Every step
@@ -24,8 +28,9 @@ from typing import Optional, Tuple
 import numpy as np
 import torch
 
-__all__ = ["get_mla_metadata", "flash_mla_with_kvcache", "device_error", "library", "LIB_PATH",
-           "PmlaError", "DEFAULT_SOFTMAX_SCALE"]
+__all__ = ["get_mla_metadata", "flash_mla_with_kvcache", "metadata_sizes", "workspace_bytes",
+           "append_kvcache", "PagePool", "absorb_query", "project_output", "device_error", "library",
+           "LIB_PATH", "PmlaError", "DEFAULT_SOFTMAX_SCALE"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedmla.so")
 PAGE_SIZE = 64
