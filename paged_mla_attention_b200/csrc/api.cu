@@ -98,10 +98,20 @@ int device_setup(int* device_out, DeviceInfo** info_out) {
   return PMLA_OK;
 }
 
+// Partial-result rows of the largest schedule for this shape, (batch + parts)
+// x h_kv x R, must stay below 2^32 so that every workspace size and offset is
+// far from overflowing (2^32 rows x 2 KB) and the counter count fits an int.
+bool too_many_rows(int batch, long long R, int h_kv) {
+  return ((long long)batch + pmla::kMaxParts) * (long long)h_kv * R > (1ll << 32);
+}
+
 int check_shape(int batch, int num_heads_per_head_k, int num_heads_k) {
   if (batch < 0 || batch > 65535) return fail(PMLA_ERR_INVALID_ARG, "batch %d not in [0, 65535]", batch);
   if (num_heads_per_head_k < 1 || num_heads_k < 1 || num_heads_k > 65535)
     return fail(PMLA_ERR_INVALID_ARG, "bad head counts (%d per KV head, %d KV heads)",
+                num_heads_per_head_k, num_heads_k);
+  if (num_heads_per_head_k > (1 << 20) || too_many_rows(batch, num_heads_per_head_k, num_heads_k))
+    return fail(PMLA_ERR_UNSUPPORTED, "shape too large (batch %d, %d rows per KV head, %d KV heads)", batch,
                 num_heads_per_head_k, num_heads_k);
   return PMLA_OK;
 }
@@ -219,7 +229,8 @@ int decode_impl(const uint16_t* q, const uint16_t* kvcache, const int32_t* block
   if (!aligned16(q) || !aligned16(kvcache) || !aligned32(o))
     return fail(PMLA_ERR_ALIGNMENT, "q and kvcache must be 16-byte aligned, o 32-byte aligned");
   const long long R = (long long)s_q * (h_q / h_kv);
-  if (R > (1 << 20)) return fail(PMLA_ERR_UNSUPPORTED, "s_q * h_q / h_kv too large");
+  if (R > (1 << 20) || too_many_rows(batch, R, h_kv))
+    return fail(PMLA_ERR_UNSUPPORTED, "s_q * h_q / h_kv too large for this batch");
   size_t lse_off;
   const size_t need = workspace_for(batch, (int)R, h_kv, num_parts, &lse_off);
   if (!workspace || workspace_bytes < need || !aligned32(workspace))

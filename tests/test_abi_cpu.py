@@ -145,3 +145,14 @@ def test_decode_with_empty_batch_is_a_no_op(lib):
     assert _decode(lib, batch=0, q=None, kv=None, bt=None, sl=None, meta=None, splits=None, o=None,
                    lse=None, ws=None, ws_bytes=0) == 0
     assert _decode(lib, batch=0, d=575) == -2       # shapes are still checked
+
+
+def test_oversized_shapes_are_rejected_before_any_size_overflows(lib):
+    P, I = ctypes.c_void_p, ctypes.c_int
+    f = lib.mla_get_metadata_sizes
+    f.argtypes = [I, I, I, P, P]
+    f.restype = I
+    parts, ws = ctypes.c_int(0), ctypes.c_size_t(0)
+    assert f(65535, 1 << 20, 65535, ctypes.byref(parts), ctypes.byref(ws)) == -2
+    assert f(1, (1 << 20) + 1, 1, ctypes.byref(parts), ctypes.byref(ws)) == -2
+    assert _decode(lib, s_q=8192, h_q=256) == -2       # R = 2^21 rows per KV head
