@@ -67,7 +67,9 @@ extern "C" {
  *       num_parts * PMLA_METADATA_INTS int32 entries, num_splits has batch+1.
  *   workspace_bytes (out): device workspace mla_decode_with_kvcache needs for
  *       split partial results of this shape (an upper bound over all lengths).
- * Uses the current CUDA device.  Errors: INVALID_ARG, UNSUPPORTED, CUDA.
+ * Uses the current CUDA device.  Errors: INVALID_ARG, UNSUPPORTED (more than
+ * 2^20 rows per KV head, or (batch + 2048) * num_heads_k * num_heads_per_head_k
+ * above 2^32), CUDA.
  */
 PMLA_API int mla_get_metadata_sizes(int batch, int num_heads_per_head_k, int num_heads_k, int* num_parts,
                            size_t* workspace_bytes);
@@ -128,9 +130,9 @@ PMLA_API int mla_get_metadata(const int32_t* cache_seqlens, int batch, int num_h
  * Alignment: q and kvcache 16-byte aligned; o and workspace 32-byte aligned.
  * batch = 0 returns PMLA_OK once the shape arguments are valid, without looking
  * at any pointer (empty tensors may be null) and without launching anything.
- * Errors: INVALID_ARG, UNSUPPORTED (d != 576, dv != 512, h_q % h_kv != 0, or
- *         h_q/h_kv neither a divisor of 128 that is >= 8 nor a multiple of 128),
- *         ALIGNMENT, WORKSPACE, CUDA.
+ * Errors: INVALID_ARG, UNSUPPORTED (d != 576, dv != 512, h_q % h_kv != 0,
+ *         h_q/h_kv neither a divisor of 128 that is >= 8 nor a multiple of 128,
+ *         or a shape mla_get_metadata_sizes rejects), ALIGNMENT, WORKSPACE, CUDA.
  * Device-side waits are bounded; a kernel that gives up records an error that
  * pmla_device_error() returns.
  * Launches: a counter-clear kernel, the decode kernel and the merge kernel, the
