@@ -355,7 +355,30 @@ def pin_unabsorbed_equals_absorbed_route(ora):
     assert np.allclose(lse, lse_lat, rtol=0, atol=1e-10)
 
 
+def pin_closed_form_golden(ora):
+    # the worked examples of golden/closed_form_cases.txt (answers in closed form,
+    # derivation in the file) to 1e-12
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "closed_form_cases.txt")
+    rows = [ln.split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    assert len(rows) == 4
+    kv = np.zeros((1, 64, 1, W.D_QK), dtype=np.float32)
+    kv[0, 0, 0, :512] = 1.0
+    kv[0, 1, 0, :512] = 2.0
+    kv[0, 1, 0, 512] = 1.0
+    kv_bits = W.f32_to_bf16_bits(kv)
+    for name, s_q, causal, scale, qi, lse_ref, o_ref in rows:
+        s_q, causal, qi = int(s_q), bool(int(causal)), int(qi)
+        q = np.zeros((1, s_q, 1, W.D_QK), dtype=np.float32)
+        q[..., 512] = 1.0
+        o, lse = ora.mla_decode(W.f32_to_bf16_bits(q), kv_bits, np.zeros((1, 1), np.int32),
+                                np.array([2], np.int32), W.D_V, causal, float(scale))
+        assert abs(lse[0, 0, qi] - float(lse_ref)) < 1e-12, name
+        assert np.all(np.abs(o[0, qi, 0] - float(o_ref)) < 1e-12), name
+
+
 ALL_PINS = [pin_bruteforce, pin_single_token, pin_equal_values, pin_page_permutation,
             pin_lse_extended, pin_zero_scale, pin_causal_reduction, pin_split_merge,
             pin_empty_rows, pin_combine_closed_form, pin_append_readback, pin_append_then_decode,
-            pin_append_overflow, pin_unabsorbed_bruteforce, pin_unabsorbed_equals_absorbed_route]
+            pin_append_overflow, pin_unabsorbed_bruteforce, pin_unabsorbed_equals_absorbed_route,
+            pin_closed_form_golden]
