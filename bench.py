@@ -2,27 +2,31 @@
 """Benchmark of the paged MLA decode hot path on B200.
 
 One *step* is one pass of the whole hot path over one batch: the length-balanced
-schedule (get_mla_metadata), the split-KV decode kernel and the merge kernel.
-The default workload is the uniform decode configuration (batch 64, s_q 1,
-128 query heads, 1 KV head, 576/512 dims, 4096 cached tokens each, 64-token
-pages in a shuffled 4096-page pool, bf16 N(0,1) data, scale 1/sqrt(192)).  Its
-inputs (302 MB of KV cache) are larger than the 126 MB L2, so no flush is
-needed between steps; the merge partials and q are small and may stay in L2.
+schedule (get_mla_metadata), the split-KV decode kernel and the merge kernel,
+replayed as one CUDA graph (the kernels form a programmatic launch chain).
 
-Prints ONE JSON line on rank 0.  ``value`` is the whole-job KV-read bandwidth
-(GB/s): KV bytes of all ranks' steps / max-over-ranks device time of the K
-timed steps.  Each step replays two CUDA graphs: the schedule, and the decode
-call (decode kernel, then the merge kernel launched as its programmatic
-dependent).  ``roofline`` reports the split-KV decode kernel, replayed alone K
-times right after the timed steps with CUDA events around each launch, against
-the measured HBM or bf16 peak; ``us_per_call`` is the decode call.  ``e2e`` times the same step through the public
-Python API from pinned host buffers (inputs copied in, o and lse copied out
-every step).  ``cpu_baseline`` times the fp64 oracle on the host cores on a
-bounded sample of the same workload.
+By default every one of the five decode workloads is timed back to back in one
+process (tiny, uniform, varlen, causal2, skew; shapes and length recipes in
+mla_workloads).  The headline line is the largest single-GPU workload, causal2
+(batch 128, two causal query tokens x 128 heads, lengths U[1024, 8192], 724 MB
+of KV), which is tensor-bound: ``value`` is its whole-job TFLOP/s per step
+(flops of all ranks' steps / max-over-ranks device time of the K timed steps).
+``per_config`` carries every workload's figures: us per step, per decode call
+and for the decode kernel alone, TFLOP/s, KV-read GB/s, the roofline bound and
+fraction, and the ncu DRAM traffic.  Workloads whose KV is larger than the
+126 MB L2 run back to back; the tiny one is timed with an L2 flush before every
+replay.
+
+``roofline`` reports the split-KV decode kernel, replayed alone min(K, 300)
+times right after the timed steps with CUDA events around each replay, against
+the measured HBM or bf16 peak; ``us_per_call`` is the decode call.  ``e2e``
+times the headline step through the public Python API from pinned host buffers
+(inputs copied in, o and lse copied out every step).  ``cpu_baseline`` times
+the fp64 oracle on the host cores on a bounded sample of the headline workload.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
     python bench.py --impl reference ...     # the oracle as the reference arm
-    python bench.py --all-configs            # one line per configuration (stderr + file)
+    python bench.py --profile --config NAME  # plain launches, for ncu
 """
 from __future__ import annotations
 
@@ -169,17 +173,25 @@ class ClockSampler:
             self.max_mhz = None
         self._stop = threading.Event()
 
+    def sample(self):
+        """One reading now (also taken at the start and the end of the timed region,
+        so that a short timed loop still records more than one sample)."""
+        if not self.ok:
+            return
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+        except Exception:
+            pass
+
     def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
-            except Exception:
-                pass
-            time.sleep(0.005)
+            self.sample()
+            time.sleep(0.002)
 
     def __enter__(self):
         if self.ok:
+            self.sample()
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
         return self
@@ -188,6 +200,7 @@ class ClockSampler:
         if self.ok:
             self._stop.set()
             self.t.join()
+            self.sample()
 
     def summary(self):
         if not self.ok:
@@ -199,14 +212,51 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- our arm
-def bench_ours(args, rank, world, local_rank):
+L2_BYTES = 126 * 1024 * 1024
+# The headline workload: the largest single-GPU configuration (batch 128, two
+# causal query tokens, 128 heads, lengths U[1024, 8192]), the compute-bound one.
+HEADLINE = "causal2"
+
+
+def timed_replays(graph, n, stream, flush_buf=None):
+    """Replays `graph` n times on `stream`; returns the per-replay times (ms) from
+    CUDA events recorded on that stream.  With `flush_buf` (larger than L2) the
+    buffer is overwritten before every replay, outside the bracketing events, so
+    each replay starts with a cold L2; without it the replays run back to back
+    (used when the inputs are larger than L2)."""
+    import torch
+    with torch.cuda.stream(stream):
+        if flush_buf is None:
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+            ev[0].record(stream)
+            for k in range(n):
+                graph.replay()
+                ev[k + 1].record(stream)
+            torch.cuda.synchronize()
+            return [ev[k].elapsed_time(ev[k + 1]) for k in range(n)]
+        ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for k in range(n):
+            flush_buf.add_(1)
+            ev0[k].record(stream)
+            graph.replay()
+            ev1[k].record(stream)
+        torch.cuda.synchronize()
+        return [ev0[k].elapsed_time(ev1[k]) for k in range(n)]
+
+
+def bench_ours(args, rank, world, local_rank, name, headline):
+    """Times one workload: K whole steps (schedule + counter clear + decode kernel +
+    merge kernel, one CUDA graph per step), then the decode kernel alone and the
+    decode call alone, each replayed min(K, 300) times with events around every
+    replay.  For the headline workload also the end-to-end run from host buffers."""
     import torch
     import paged_mla_attention_b200 as pm
     sys.path.insert(0, os.path.join(ROOT, "tests"))
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = W.WORKLOADS[args.config]
+    w = W.WORKLOADS[name]
     inp = rank_inputs(w, rank)   # weak scaling: each rank its own batch
     wc = work_counts(inp)
     peaks, peaks_src = load_peaks()
@@ -231,8 +281,7 @@ def bench_ours(args, rank, world, local_rank):
 
     def step_decode(stage="all"):
         pm.flash_mla_with_kvcache(d["q"], d["kvcache"], d["block_table"], d["cache_seqlens"], W.D_V,
-                                  meta_holder["m"], meta_holder["s"],
-                                  softmax_scale=inp["softmax_scale"], causal=inp["causal"],
+                                  meta_holder["m"], meta_holder["s"], inp["causal"], inp["softmax_scale"],
                                   out=(o, lse), workspace=ws, stage=stage)
 
     if args.profile:
@@ -246,7 +295,11 @@ def bench_ours(args, rank, world, local_rank):
             raise RuntimeError(f"device error {err}")
         return None, inp, wc
 
-    # warm-up (also compiles nothing: the library is prebuilt)
+    # inputs that fit in L2 (the tiny parity workload) are timed with an L2 flush
+    # before every replay; the others are larger than L2 and run back to back
+    flush_buf = (torch.zeros((2 * L2_BYTES // 4,), dtype=torch.int32, device=dev)
+                 if wc["kv_bytes"] < 2 * L2_BYTES else None)
+
     stream = torch.cuda.Stream(dev)
     stream.wait_stream(torch.cuda.current_stream(dev))
     with torch.cuda.stream(stream):
@@ -274,80 +327,86 @@ def bench_ours(args, rank, world, local_rank):
     with torch.cuda.graph(g_step, stream=stream):
         step_meta()
         step_decode("all")
-    for _ in range(3):
-        g_meta.replay()  # fills the schedule that g_all and g_dec read
-        g_step.replay()
-        g_all.replay()
-        g_dec.replay()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g_meta.replay()  # fills the schedule that g_all and g_dec read
+            g_step.replay()
+            g_all.replay()
+            g_dec.replay()
     torch.cuda.synchronize(dev)
 
     K = args.steps
-    ev_start = torch.cuda.Event(enable_timing=True)
-    ev_end = torch.cuda.Event(enable_timing=True)
     KA = min(K, 300)
-    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(KA + 1)]
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local_rank) as clk:
-        ev_start.record()
-        for k in range(K):
-            g_step.replay()
-        ev_end.record()
-        torch.cuda.synchronize(dev)
-        # the decode kernel alone, then the decode call alone: KA more launches each
+        if flush_buf is None:
+            with torch.cuda.stream(stream):
+                ev_start = torch.cuda.Event(enable_timing=True)
+                ev_end = torch.cuda.Event(enable_timing=True)
+                ev_start.record(stream)
+                for k in range(K):
+                    g_step.replay()
+                ev_end.record(stream)
+            torch.cuda.synchronize(dev)
+            elapsed_ms = ev_start.elapsed_time(ev_end)
+        else:
+            elapsed_ms = float(np.sum(timed_replays(g_step, K, stream, flush_buf)))
+        clk.sample()
+        # the decode kernel alone, then the decode call alone: KA more replays each
         # right after the timed steps (same stream, same inputs), each bracketed by
         # events; KA is capped so that these runs add little heat after long step loops
-        ev_c = [torch.cuda.Event(enable_timing=True) for _ in range(KA + 1)]
-        ev_c[0].record()
-        for k in range(KA):
-            g_dec.replay()
-            ev_c[k + 1].record()
-        torch.cuda.synchronize(dev)
-        ev_a[0].record()
-        for k in range(KA):
-            g_all.replay()
-            ev_a[k + 1].record()
-        torch.cuda.synchronize(dev)
+        dec_ms = float(np.mean(timed_replays(g_dec, KA, stream, flush_buf)))   # clear + decode kernel
+        call_ms = float(np.mean(timed_replays(g_all, KA, stream, flush_buf)))  # clear + decode + merge
     if world > 1:
         dist.barrier()
-    elapsed_ms = ev_start.elapsed_time(ev_end)
-    call_ms = float(np.mean([ev_a[k].elapsed_time(ev_a[k + 1]) for k in range(KA)]))  # clear + decode + merge
-    dec_ms = float(np.mean([ev_c[k].elapsed_time(ev_c[k + 1]) for k in range(KA)]))  # clear + decode kernel
     err = pm.device_error()
     if err:
         raise RuntimeError(f"device error {err} in the timed region")
     elapsed_ms = max_over_ranks(elapsed_ms, dev)
 
-    # end-to-end through the public API from pinned host buffers
-    e2e_steps = max(3, min(K, args.e2e_steps))
-    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+    t_roof, bound = roofline_time(wc, peaks)
+    per_step_s = elapsed_ms / 1e3 / K
+    if bound == "tensor":
+        value, unit = world * wc["flops"] / per_step_s / 1e12, "TFLOP/s"
+    else:
+        value, unit = whole_job_gbs(world, wc["kv_bytes"], per_step_s), "GB/s"
 
-    def e2e_step():
-        dd = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
-        m, s = pm.get_mla_metadata(dd["cache_seqlens"], R, inp["h_kv"])
-        oo, ll = pm.flash_mla_with_kvcache(dd["q"], dd["kvcache"], dd["block_table"],
-                                           dd["cache_seqlens"], W.D_V, m, s,
-                                           softmax_scale=inp["softmax_scale"], causal=inp["causal"])
-        o_h.copy_(oo, non_blocking=True)
-        lse_h.copy_(ll, non_blocking=True)
+    e2e = None
+    if headline:
+        # end-to-end through the public API from pinned host buffers
+        e2e_steps = max(3, min(K, args.e2e_steps))
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
 
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(e2e_steps):
+        def e2e_step():
+            dd = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+            m, s = pm.get_mla_metadata(dd["cache_seqlens"], R, inp["h_kv"])
+            oo, ll = pm.flash_mla_with_kvcache(dd["q"], dd["kvcache"], dd["block_table"],
+                                               dd["cache_seqlens"], W.D_V, m, s, inp["causal"],
+                                               inp["softmax_scale"])
+            o_h.copy_(oo, non_blocking=True)
+            lse_h.copy_(ll, non_blocking=True)
+
         e2e_step()
-    e1.record()
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    e2e_ms = max_over_ranks(e2e_ms, dev)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+        e2e_s = e2e_ms / 1e3 / e2e_steps
+        e2e_v = (world * wc["flops"] / e2e_s / 1e12) if unit == "TFLOP/s" else (world * wc["kv_bytes"] / e2e_s / 1e9)
+        e2e = {"value": round(e2e_v, 3), "unit": unit, "steps": e2e_steps, "ms_per_step": round(e2e_s * 1e3, 4),
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     # correctness spot-check of this very run against the oracle (rank 0, two sequences)
     spot = None
@@ -361,49 +420,61 @@ def bench_ours(args, rank, world, local_rank):
         lg = lse.cpu().numpy()[seqs][:, ::8].astype(np.float64)
         spot = compare(og, lg, ro, rl, what="bench spot check")
 
-    per_step_s = elapsed_ms / 1e3 / K
-    value = whole_job_gbs(world, wc["kv_bytes"], per_step_s)
     dec_s = dec_ms / 1e3
-    t_roof, bound = roofline_time(wc, peaks)
     if bound == "hbm":
         achieved = wc["bytes"] / dec_s / 1e9
-        peak, unit = peaks["hbm_gbs"], "GB/s"
+        peak, runit = peaks["hbm_gbs"], "GB/s"
     else:
         achieved = wc["flops"] / dec_s / 1e12
-        peak, unit = peaks["bf16_tflops"], "TFLOP/s"
+        peak, runit = peaks["bf16_tflops"], "TFLOP/s"
+    l2 = ("inputs fit in L2: L2 flushed (256 MB write) before every timed replay" if flush_buf is not None
+          else f"inputs ({wc['kv_bytes'] / 1e6:.0f} MB KV) larger than the 126 MB L2; no flush")
     result = {
-        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(elapsed_ms / K, 6), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": workload_desc(w), "global_batch": inp["batch"] * world,
                    "kv_tokens_per_gpu": wc["tokens"], "parallelism": f"replicas x{world} (batch-sharded, no exchange)",
-                   "l2": "inputs (302 MB KV) larger than the 126 MB L2; no flush",
+                   "l2": l2,
                    "step": "schedule + counter clear + split-KV decode + merge, one CUDA graph per step"},
         "us_decode_kernel": round(dec_ms * 1e3, 3),
         "us_per_call": round(call_ms * 1e3, 3),
         "tflops": round(wc["flops"] / dec_s / 1e12, 2),
+        "tflops_per_call": round(wc["flops"] / (call_ms / 1e3) / 1e12, 2),
         "kv_read_gbs_per_call": round(wc["kv_bytes"] / (call_ms / 1e3) / 1e9, 1),
-        "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+        "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": runit,
                      "frac": round(achieved / peak, 4), "traffic": (args.traffic if args.traffic is not None
-                                                               else measured_traffic(args.config)),
+                                                               else measured_traffic(name)),
                      "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "kernel": "split-KV decode kernel (timed alone; the merge kernel follows it)",
                      "peak_source": f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback",
+                     "algorithmic_bytes": wc["bytes"], "algorithmic_flops": wc["flops"],
                      "roofline_us": round(t_roof * 1e6, 2),
                      "frac_of_roofline_time": round(t_roof / dec_s, 4)},
-        "e2e": {"value": round(world * wc["kv_bytes"] / (e2e_ms / 1e3 / e2e_steps) / 1e9, 3), "unit": "GB/s",
-                "steps": e2e_steps, "ms_per_step": round(e2e_ms / e2e_steps, 4),
-                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": 4 * K,  # schedule, counter clear, decode, merge per timed step
         "clocks": clk.summary(),
     }
+    if e2e is not None:
+        result["e2e"] = e2e
     if spot is not None:
         result["parity_spot_check"] = {k: float(f"{v:.4g}") for k, v in spot.items()}
     return result, inp, wc
 
 
-def cpu_baseline(inp, wc, budget_s):
-    """The oracle as it stands, on the host cores, on a bounded sample of the workload."""
+def config_summary(res: dict) -> dict:
+    """The per-workload figures carried in the headline line's per_config object."""
+    r = res["roofline"]
+    return {"workload": res["config"]["workload"], "us_per_step": round(res["ms_per_step"] * 1e3, 3),
+            "us_per_call": res["us_per_call"], "us_decode_kernel": res["us_decode_kernel"],
+            "tflops": res["tflops"], "kv_read_gbs": round(res["kv_read_gbs_per_call"], 1),
+            "bound": r["bound"], "achieved": r["achieved"], "peak": r["peak"], "unit": r["unit"],
+            "frac": r["frac"], "roofline_us": r["roofline_us"], "traffic": r["traffic"],
+            "l2": res["config"]["l2"], "clocks": res["clocks"]}
+
+
+def cpu_baseline(inp, wc, budget_s, unit="GB/s"):
+    """The oracle as it stands, on the host cores, on a bounded sample of the workload,
+    in the headline's unit (KV GB/s, or TFLOP/s for a tensor-bound workload)."""
     import oracle
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     from gpu_helpers import subset
@@ -419,8 +490,8 @@ def cpu_baseline(inp, wc, budget_s):
         if t_total >= budget_s:
             break
     frac = done_tokens / max(wc["tokens"], 1)
-    value = frac * wc["kv_bytes"] / t_total / 1e9
-    return {"value": round(value, 5), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+    value = frac * (wc["flops"] / 1e12 if unit == "TFLOP/s" else wc["kv_bytes"] / 1e9) / t_total
+    return {"value": round(value, 8), "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{seqs_done} of {inp['batch']} sequences (all heads, all tokens), "
                       f"{frac:.3f} of the workload's KV-token work, fp64, {t_total:.1f} s"}
 
@@ -431,9 +502,11 @@ def bench_reference(args):
     import oracle
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     from gpu_helpers import subset
-    w = W.WORKLOADS[args.config]
+    w = W.WORKLOADS[args.config or HEADLINE]
     inp = W.make_inputs(w)
     wc = work_counts(inp)
+    peaks, _ = load_peaks()
+    unit = "TFLOP/s" if roofline_time(wc, peaks)[1] == "tensor" else "GB/s"
     # size each step so that warm-up + timed steps take about `budget` seconds
     probe = subset(inp, [0], [0, 1])
     t = time.perf_counter()
@@ -456,18 +529,18 @@ def bench_reference(args):
         tt += dt
         work += wk
     frac = work / (wc["tokens"] * inp["h_q"])
-    value = frac * wc["kv_bytes"] / tt / 1e9
+    value = frac * (wc["flops"] / 1e12 if unit == "TFLOP/s" else wc["kv_bytes"] / 1e9) / tt
     sample = (f"each step: 1 sequence x {heads} of {inp['h_q']} heads (all tokens); "
               f"{frac:.4f} of one workload's row-token work in total, fp64")
     return {
-        "metric": METRIC, "value": round(value, 6), "unit": "GB/s", "n_gpus": args.gpus,
+        "metric": METRIC, "value": round(value, 8), "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tt / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
         "config": {"workload": workload_desc(w), "global_batch": inp["batch"]},
-        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": oracle.num_threads(),
+        "cpu_baseline": {"value": round(value, 8), "unit": unit, "cores": oracle.num_threads(),
                          "kind": "oracle", "sample": sample},
-        "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+        "e2e": {"value": round(value, 8), "unit": unit, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -580,9 +653,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="uniform", choices=list(W.WORKLOADS))
-    ap.add_argument("--all-configs", action="store_true",
-                    help="bench every configuration; one JSON line each on stderr and in --out")
+    ap.add_argument("--config", default=None, choices=list(W.WORKLOADS),
+                    help="bench this workload only (default: all five, headline " + HEADLINE + ")")
     ap.add_argument("--out", default=None)
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
@@ -626,29 +698,31 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     try:
         if args.profile:
-            bench_ours(args, rank, world, local_rank)
+            bench_ours(args, rank, world, local_rank, args.config or HEADLINE, False)
             if rank == 0:
-                print(json.dumps({"profile_run": args.config, "steps": args.steps, "warmup": args.warmup}))
+                print(json.dumps({"profile_run": args.config or HEADLINE, "steps": args.steps,
+                                  "warmup": args.warmup}))
             return
-        configs = list(W.WORKLOADS) if args.all_configs else [args.config]
-        main_name = "uniform" if args.all_configs else args.config
-        lines, main = [], None
+        # every workload back to back in one process (or the one --config names);
+        # the headline line is the largest workload, with the others in per_config
+        headline = args.config or HEADLINE
+        configs = [args.config] if args.config else list(W.WORKLOADS)
+        per_config, main = {}, None
         for name in configs:
-            args.config = name
-            res, inp, wc = bench_ours(args, rank, world, local_rank)
-            lines.append(res)
-            if name == main_name:
+            res, inp, wc = bench_ours(args, rank, world, local_rank, name, name == headline)
+            per_config[name] = config_summary(res)
+            if name == headline:
                 main = (res, inp, wc)
-            if args.all_configs and rank == 0:
+            if rank == 0:
                 log(json.dumps(res))
         res, inp, wc = main
+        res["per_config"] = per_config
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            res["cpu_baseline"] = cpu_baseline(inp, wc, args.cpu_budget)
+            res["cpu_baseline"] = cpu_baseline(inp, wc, args.cpu_budget, res["unit"])
         if rank == 0:
             if args.out:
                 with open(args.out, "w") as f:
-                    for r in lines:
-                        f.write(json.dumps(r) + "\n")
+                    f.write(json.dumps(res) + "\n")
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:

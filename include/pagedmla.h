@@ -53,6 +53,22 @@ extern "C" {
 #define PMLA_ERR_DEVICE (-6)       /* a kernel reported an error (see below)           */
 #define PMLA_ERR_EXHAUSTED (-7)    /* the page pool has fewer free pages than asked    */
 
+/* The same status codes under the mla_ prefix of the decode calls. */
+#define MLA_OK PMLA_OK
+#define MLA_ERR_INVALID_ARG PMLA_ERR_INVALID_ARG
+#define MLA_ERR_UNSUPPORTED PMLA_ERR_UNSUPPORTED
+#define MLA_ERR_ALIGNMENT PMLA_ERR_ALIGNMENT
+#define MLA_ERR_CUDA PMLA_ERR_CUDA
+#define MLA_ERR_WORKSPACE PMLA_ERR_WORKSPACE
+#define MLA_ERR_DEVICE PMLA_ERR_DEVICE
+#define MLA_ERR_EXHAUSTED PMLA_ERR_EXHAUSTED
+
+/* Codes the kernels record in the device error word (pmla_device_error()). */
+#define PMLA_DEVERR_BAD_PAGE 2    /* a block_table entry outside [0, num_pages): read as zeros  */
+#define PMLA_DEVERR_BAD_APPEND 3  /* an appended row lies past its sequence's block table        */
+#define PMLA_DEVERR_BAD_SEQLEN 4  /* cache_seqlens[b] > 64 * max_pages_per_seq: decoded as empty */
+#define PMLA_DEVERR_WAIT_BASE 100 /* + id of a bounded device wait that gave up                  */
+
 #define PMLA_PAGE_SIZE 64     /* tokens per KV page                                  */
 #define PMLA_HEAD_DIM 576     /* q / k width: 512 latent (c^KV) + 64 RoPE (k^R)      */
 #define PMLA_HEAD_DIM_V 512   /* value width: the latent part of the same row        */
@@ -118,7 +134,10 @@ PMLA_API int mla_get_metadata(const int32_t* cache_seqlens, int batch, int num_h
  *   kvcache       bf16 [num_pages][64][h_kv][576]
  *   block_table   int32 [batch][max_pages_per_seq]; entries for pages a
  *                 sequence uses must lie in [0, num_pages)
- *   cache_seqlens int32 [batch], each <= 64 * max_pages_per_seq
+ *   cache_seqlens int32 [batch], each <= 64 * max_pages_per_seq; a longer
+ *                 sequence is not read at all: its rows are written as empty
+ *                 (o = 0, lse = -inf) and the device error word records
+ *                 PMLA_DEVERR_BAD_SEQLEN
  *   tile_scheduler_metadata, num_parts, num_splits: from mla_get_metadata on
  *                 the same cache_seqlens and shape (must not be modified
  *                 before this call has run on the device)
@@ -287,12 +306,16 @@ PMLA_API int mla_project_output(const uint16_t* o_latent, const uint16_t* w_uv, 
 /*
  * Reads and clears the device error word of the current device (synchronises
  * the device).  Returns 0 if no kernel reported an error since the last call,
- * else the kernel's error code (a positive number naming the wait that gave up).
+ * else the first code a kernel recorded (PMLA_DEVERR_*; PMLA_DEVERR_WAIT_BASE
+ * plus an id names a bounded wait that gave up).
  */
 PMLA_API int pmla_device_error(void);
 
 /* Message for the last failing call of this host thread ("" if none). */
 PMLA_API const char* pmla_last_error(void);
+
+/* The same message under the mla_ prefix of the decode calls. */
+PMLA_API const char* mla_get_last_error(void);
 
 /* Library version string. */
 PMLA_API const char* pmla_version(void);

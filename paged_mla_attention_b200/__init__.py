@@ -89,6 +89,8 @@ def _load() -> ctypes.CDLL:
     lib.pmla_device_error.restype = I
     lib.pmla_last_error.argtypes = []
     lib.pmla_last_error.restype = ctypes.c_char_p
+    lib.mla_get_last_error.argtypes = []
+    lib.mla_get_last_error.restype = ctypes.c_char_p
     lib.pmla_version.argtypes = []
     lib.pmla_version.restype = ctypes.c_char_p
     return lib
@@ -167,20 +169,25 @@ def get_mla_metadata(cache_seqlens: torch.Tensor, num_heads_per_head_k: int,
 def flash_mla_with_kvcache(q: torch.Tensor, kvcache: torch.Tensor, block_table: torch.Tensor,
                            cache_seqlens: torch.Tensor, head_dim_v: int,
                            tile_scheduler_metadata: torch.Tensor, num_splits: torch.Tensor,
-                           softmax_scale: Optional[float] = None, causal: bool = False,
+                           causal: bool = False, softmax_scale: Optional[float] = None, *,
                            out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
                            workspace: Optional[torch.Tensor] = None, stage: str = "all"
                            ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Paged MLA decode.
+
+    The positional order is the one of the FlashMLA usage call (usage step 4):
+    q, kvcache, block_table, cache_seqlens, dv, tile_scheduler_metadata,
+    num_splits, causal; softmax_scale follows it.
 
     q           bf16 [batch, s_q, h_q, 576]
     kvcache     bf16 [num_pages, 64, h_kv, 576]
     block_table int32 [batch, max_pages]
     cache_seqlens int32 [batch]
     head_dim_v  512
+    causal      mask query token i of s_q to cached tokens j <= seqlen - s_q + i
     Returns o bf16 [batch, s_q, h_q, 512] and lse fp32 [batch, h_q, s_q] (natural log).
-    softmax_scale defaults to 1/sqrt(192).  ``out`` and ``workspace`` may be
-    passed to avoid per-call allocation.  ``stage`` selects the C entry point:
+    softmax_scale defaults to 1/sqrt(192).  ``out`` and ``workspace`` (keyword
+    only) may be passed to avoid per-call allocation.  ``stage`` selects the C entry point:
     "all" (mla_decode_with_kvcache), "decode" (mla_decode_splits, the decode
     kernel alone) or "merge" (mla_merge_splits, the merge kernel alone; pass the
     same ``out`` and ``workspace`` as the "decode" call).

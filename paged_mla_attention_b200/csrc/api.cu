@@ -155,6 +155,8 @@ const char* pmla_version(void) { return "pagedmla 0.1.0 (sm_100a)"; }
 
 const char* pmla_last_error(void) { return g_last_error.c_str(); }
 
+const char* mla_get_last_error(void) { return g_last_error.c_str(); }
+
 int mla_get_metadata_sizes(int batch, int num_heads_per_head_k, int num_heads_k, int* num_parts,
                            size_t* workspace_bytes) {
   g_last_error.clear();
@@ -335,6 +337,8 @@ int decode_impl(const uint16_t* q, const uint16_t* kvcache, const int32_t* block
   const pmla::WorkspaceLayout wl2 = pmla::workspace_layout(batch, (int)R, h_kv, num_parts);
   pmla::CombineParams c;
   c.num_splits = num_splits;
+  c.seqlens = cache_seqlens;
+  c.max_pages = max_pages_per_seq;
   c.part_o = static_cast<float*>(workspace);
   c.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + wl2.lse_off);
   c.seq_done = reinterpret_cast<const int*>(static_cast<char*>(workspace) + wl2.done_off);

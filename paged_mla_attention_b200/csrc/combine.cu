@@ -6,7 +6,8 @@
 //   lse = log sum_k exp(lse_k),   o = sum_k exp(lse_k - lse) o_k,
 // computed with the largest lse_k subtracted first.  Empty pieces
 // (lse_k = -inf) weigh nothing; if every piece is empty, o = 0, lse = -inf.
-// Sequences with no pages at all (n = 0) also get o = 0, lse = -inf here;
+// Sequences with no pages at all (n = 0), and sequences longer than their
+// block table (skipped by the decode kernel), also get o = 0, lse = -inf here;
 // unsplit sequences (n = 1) were written by the decode kernel directly.
 //
 // Layout: the partials are chunk-major, [slot][h_kv][64 chunks of 8 columns]
@@ -61,7 +62,9 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombinePar
   const int r0 = (blockIdx.x / kQuarters) * kMergeRows;
   const int quarter = blockIdx.x % kQuarters;
   const int s0 = P.num_splits[b];
-  const int n = P.num_splits[b + 1] - s0;
+  // a sequence longer than its block table was skipped by the decode kernel
+  // (which recorded the error): its rows are written here as empty
+  const int n = (long long)P.seqlens[b] > (long long)P.max_pages * kPage ? 0 : P.num_splits[b + 1] - s0;
   const bool last_block =
       blockIdx.x == gridDim.x - 1 && blockIdx.y == gridDim.y - 1 && blockIdx.z == gridDim.z - 1;
   if (n == 1) {  // written by the decode kernel directly

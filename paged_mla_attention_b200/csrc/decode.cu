@@ -168,11 +168,22 @@ __device__ __forceinline__ int seq_pages(const DecodeParams& P, int b) {
   return n < P.max_pages ? n : P.max_pages;
 }
 
+// A sequence longer than its block table (cache_seqlens[b] > 64 * max_pages)
+// is skipped by every role alike -- nothing of it is read -- and recorded in
+// the device error word; the merge kernel writes its rows as empty.
+__device__ __forceinline__ bool seq_too_long(const DecodeParams& P, int b) {
+  return (long long)P.seqlens[b] > (long long)P.max_pages * kPage;
+}
+
 template <class F>
 __device__ __forceinline__ void for_each_piece(const DecodeParams& P, const PartIter& it, F&& f) {
   const int last = min(it.b1, P.batch - 1);
   for (int k = 0; k <= last - it.b0; ++k) {
     const int b = it.rev ? last - k : it.b0 + k;
+    if (seq_too_long(P, b)) {
+      if (threadIdx.x == 0) atomicCAS(P.err, 0, kErrBadSeqlen);
+      continue;
+    }
     const int n = seq_pages(P, b);
     const int p0 = (b == it.b0) ? min(it.pg0, n) : 0;
     const int p1 = (b == it.b1) ? min(max(it.pg1, 0), n) : n;

@@ -27,6 +27,7 @@ enum DeviceError : int {
   kErrBadSmemAlign = 1,
   kErrBadPage = 2,
   kErrBadAppend = 3,   // an appended token lies past the sequence's block table
+  kErrBadSeqlen = 4,   // cache_seqlens[b] > 64 * max_pages: the sequence is treated as empty
   kErrWaitBase = 100,  // + the id of the wait that gave up
 };
 
@@ -52,13 +53,14 @@ struct DecodeParams {
 
 struct CombineParams {
   const int32_t* num_splits;
+  const int32_t* seqlens;       // [b]: a sequence longer than its block table merges as empty
   const float* part_o;
   const float* part_lse;
   const int* seq_done;          // [b][h_kv][n_rg]: 2 signals per finished split piece
   int* err;                     // device error word
   uint16_t* o;
   float* lse;
-  int batch, s_q, h_q, h_kv, hpk, R, n_rg, num_parts;
+  int batch, s_q, h_q, h_kv, hpk, R, n_rg, num_parts, max_pages;
 };
 
 struct AppendParams {

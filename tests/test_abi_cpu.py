@@ -156,3 +156,23 @@ def test_oversized_shapes_are_rejected_before_any_size_overflows(lib):
     assert f(65535, 1 << 20, 65535, ctypes.byref(parts), ctypes.byref(ws)) == -2
     assert f(1, (1 << 20) + 1, 1, ctypes.byref(parts), ctypes.byref(ws)) == -2
     assert _decode(lib, s_q=8192, h_q=256) == -2       # R = 2^21 rows per KV head
+
+
+def test_mla_get_last_error_is_the_same_message(lib):
+    lib.pmla_last_error.restype = ctypes.c_char_p
+    lib.mla_get_last_error.restype = ctypes.c_char_p
+    assert _decode(lib, d=575) == -2
+    assert lib.mla_get_last_error() == lib.pmla_last_error() and b"576" in lib.mla_get_last_error()
+
+
+def test_binding_follows_the_usage_call_order():
+    # FlashMLA usage step 4: (q, kvcache, block_table, cache_seqlens, dv,
+    # tile_scheduler_metadata, num_splits, causal); softmax_scale after it and the
+    # buffers/stage selector keyword-only, so a positional causal cannot land elsewhere
+    import inspect
+    from paged_mla_attention_b200 import flash_mla_with_kvcache
+    ps = list(inspect.signature(flash_mla_with_kvcache).parameters.values())
+    assert [p.name for p in ps[:9]] == ["q", "kvcache", "block_table", "cache_seqlens", "head_dim_v",
+                                        "tile_scheduler_metadata", "num_splits", "causal", "softmax_scale"]
+    assert all(p.kind == p.POSITIONAL_OR_KEYWORD for p in ps[:9])
+    assert all(p.kind == p.KEYWORD_ONLY for p in ps[9:])
