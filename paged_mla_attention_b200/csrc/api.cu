@@ -57,7 +57,8 @@ bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) ==
 
 struct DeviceInfo {
   bool ready = false;
-  int max_clusters = 0;
+  int max_clusters = 0;       // 2-CTA decode clusters resident at once
+  int max_clusters_pair = 0;  // 4-CTA decode clusters (two row groups each) resident at once
   int* err_ptr = nullptr;
 };
 std::mutex g_mu;
@@ -82,14 +83,16 @@ int device_setup(int* device_out, DeviceInfo** info_out) {
     if ((size_t)prop.sharedMemPerBlockOptin < pmla::decode_smem_bytes())
       return fail(PMLA_ERR_UNSUPPORTED, "device offers %zu B shared memory per block, need %zu",
                   (size_t)prop.sharedMemPerBlockOptin, pmla::decode_smem_bytes());
-    int n = 0;
-    int rc = pmla::decode_max_active_clusters(dev, &n);
+    int n = 0, n4 = 0;
+    int rc = pmla::decode_max_active_clusters(dev, false, &n);
+    if (rc == 0) rc = pmla::decode_max_active_clusters(dev, true, &n4);
     if (rc != 0) return fail_cuda((cudaError_t)rc, "cudaOccupancyMaxActiveClusters");
-    if (n < 1) return fail(PMLA_ERR_UNSUPPORTED, "decode kernel cannot be resident on this device");
+    if (n < 1 || n4 < 1) return fail(PMLA_ERR_UNSUPPORTED, "decode kernel cannot be resident on this device");
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_device_error);
     if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress(device error word)");
     d.max_clusters = n;
+    d.max_clusters_pair = n4;
     d.err_ptr = static_cast<int*>(p);
     d.ready = true;
   }
@@ -116,10 +119,14 @@ int check_shape(int batch, int num_heads_per_head_k, int num_heads_k) {
   return PMLA_OK;
 }
 
+// Scheduler parts: as many (part, KV head, cluster) work units as decode clusters
+// fit on the device at once.  A KV head with one 128-row group takes one 2-CTA
+// cluster per part; with more, one 4-CTA cluster per two row groups.
 int parts_for(const DeviceInfo& d, int num_heads_per_head_k, int num_heads_k) {
   const int n_rg = (num_heads_per_head_k + pmla::kRows - 1) / pmla::kRows;
-  const long long groups = (long long)n_rg * num_heads_k;
-  long long parts = d.max_clusters / groups;
+  const bool pair = pmla::decode_uses_pairs(n_rg);
+  const long long groups = (long long)(pair ? (n_rg + 1) / 2 : n_rg) * num_heads_k;
+  long long parts = (pair ? d.max_clusters_pair : d.max_clusters) / groups;
   return (int)(parts < 1 ? 1 : parts);
 }
 
@@ -280,6 +287,22 @@ int decode_impl(const uint16_t* q, const uint16_t* kvcache, const int32_t* block
         return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled (value tiles) failed (%d)", (int)cr);
   }
 
+    // the same 4-D view with boxes of 2 column chunks (16 KB): the pair variant's
+    // page stages and value halves
+    CUtensorMap tmap_kv2;
+    {
+      cuuint64_t vdim[4] = {64, (cuuint64_t)num_pages * pmla::kPage, (cuuint64_t)pmla::kD / 64,
+                            (cuuint64_t)h_kv};
+      cuuint64_t vstride[3] = {(cuuint64_t)h_kv * pmla::kD * 2, 128, (cuuint64_t)pmla::kD * 2};
+      cuuint32_t vbox[4] = {64, (cuuint32_t)pmla::kPage, 2, 1};
+      cuuint32_t vestride[4] = {1, 1, 1, 1};
+      cr = encode(&tmap_kv2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t*>(kvcache), vdim,
+                  vstride, vbox, vestride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (cr != CUDA_SUCCESS)
+        return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled (two-chunk tiles) failed (%d)", (int)cr);
+    }
+
     // q as a 2-D tensor: [576 columns] x [batch*s_q*h_q rows]; boxes of 64 columns
     // x min(h_q/h_kv, 128) rows with the 128-byte swizzle.
     CUtensorMap tmap_q;
@@ -321,7 +344,8 @@ int decode_impl(const uint16_t* q, const uint16_t* kvcache, const int32_t* block
     p.num_pages = num_pages;
     p.causal = causal ? 1 : 0;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
-    if ((long long)num_parts * h_kv * p.n_rg > (1ll << 30))
+    const bool pair = pmla::decode_uses_pairs(p.n_rg);
+    if ((long long)num_parts * h_kv * p.n_rg > (1ll << 28))
       return fail(PMLA_ERR_UNSUPPORTED, "grid too large");
 
     cudaError_t e = pmla::decode_prepare(dev);
@@ -329,7 +353,7 @@ int decode_impl(const uint16_t* q, const uint16_t* kvcache, const int32_t* block
     // the merge kernel counts completion signals from zero
     e = pmla::launch_clear_counters(p.seq_done, (int)wl.done_count, st);
     if (e != cudaSuccess) return fail_cuda(e, "clearing the completion counters");
-    e = pmla::launch_decode(p, tmap, tmap_q, tmap_v, st);
+    e = pmla::launch_decode(p, tmap, tmap_q, tmap_v, tmap_kv2, pair, st);
     if (e != cudaSuccess) return fail_cuda(e, "decode kernel launch");
   }
   if (!(stages & kStageMerge)) return PMLA_OK;

@@ -40,6 +40,26 @@
 //     max, and run the epilogue (O / l -> bf16 o, or fp32 partials) at the end
 //     of each piece.
 //
+// Pair variant (two or more row groups per KV head, e.g. two query tokens x 128
+// heads): the two 128-row groups of a (sequence, part) read the same pages, so
+// they share one 4-CTA cluster built from two CTA pairs (cta_group::2) instead
+// of two independent clusters:
+//   ranks 0, 1 (S pair): each CTA holds the query of its own row group in TMEM
+//     and streams only its own page of each page pair from HBM (rank 0 page A,
+//     rank 1 page B, chunk stages of 16 KB = two 64-column chunks); one thread
+//     of rank 0 issues M = 256 score MMAs whose B operand (the 128 tokens of the
+//     pair) is split between the two CTAs' shared memory, so every page byte
+//     enters one SM once and feeds both tensor cores.  Each CTA's softmax
+//     warpgroups then work on their own 128 rows exactly as above and send P
+//     to the O-CTA of their row group (rank + 2).
+//   ranks 2, 3 (O pair): each loads only its half of the value columns of each
+//     page ({0,1,4,5} or {2,3,6,7} of the eight 64-column chunks); one thread
+//     of rank 2 issues M = 256 (both row groups) by N = 256 MMAs whose B operand
+//     (the value tile) is split the same way; each CTA keeps its row group's
+//     128 x 512 accumulator.  Rescale and epilogue commands go to both CTAs.
+// Compared with two independent clusters this halves the bytes each page puts
+// through shared memory and the B-operand shared-memory reads per MMA.
+//
 // Launch: a programmatic dependent of the counter-clear kernel (setup overlaps
 // the kernels before it; the schedule is read after griddepcontrol.wait); its
 // own dependent, the merge kernel, may start as soon as every CTA is resident.
@@ -92,9 +112,10 @@ enum : int {
   kBarVFull = kBarStageFree + kStageBufs,  // O [4] V half-stage loaded (TMA tx)
   kBarVEmpty = kBarVFull + kVStages,     // O [4] V half-stage consumed (commit)
   kBarPFull = kBarVEmpty + kVStages,     // O [kPSlots] P slot written (armed + bulk-copy tx)
-  kBarPCons = kBarPFull + kPSlots,       // O [kPSlots] P slot consumed (commit + 8 warps)
-  kBarCmdFull = kBarPCons + kPSlots,     // O mailbox command posted (1)
-  kBarCmdDone = kBarCmdFull + 1,         // O command done (256)
+  kBarPCons = kBarPFull + kPSlots,       // O [kPSlots] P slot consumed (commit + 8 warps; pair: + 8 of the mate)
+  kBarPeerP = kBarPCons + kPSlots,       // O [kPSlots] pair: the mate O-CTA's P slot landed (remote arrival)
+  kBarCmdFull = kBarPeerP + kPSlots,     // O mailbox command posted (1)
+  kBarCmdDone = kBarCmdFull + 1,         // O command done (256; pair: 1 per O-CTA, on rank 2)
   kBarDrain = kBarCmdDone + 1,           // both: all issued MMAs complete
   kNumBars = kBarDrain + 1
 };
@@ -208,6 +229,8 @@ __device__ __forceinline__ int load_page(const DecodeParams& P, int b, int p) {
 
 // TMA the 64-column chunk c of this tile's 128 query rows into `dst`
 // (boxes of min(hpk,128) rows; rows past R are left untouched).  Returns bytes.
+// kPairLoad: the bytes complete on `bar`, a barrier of either CTA of the pair.
+template <bool kPairLoad = false>
 __device__ __forceinline__ uint32_t load_q_chunk(const DecodeParams& P, const CUtensorMap* tmap_q,
                                                  uint32_t dst, uint32_t bar, int b, int g, int rg,
                                                  int c, uint64_t pol, bool issue) {
@@ -219,16 +242,32 @@ __device__ __forceinline__ uint32_t load_q_chunk(const DecodeParams& P, const CU
     if (issue) {
       const int qi = rr0 / P.hpk;
       const int row = (b * P.s_q + qi) * P.h_q + g * P.hpk + rr0 % P.hpk;
-      tma_load_2d(dst + (uint32_t)(j * qbox * 128), tmap_q, bar, c * 64, row, pol);
+      if constexpr (kPairLoad)
+        tma_load_2d_pair(dst + (uint32_t)(j * qbox * 128), tmap_q, bar, c * 64, row, pol);
+      else
+        tma_load_2d(dst + (uint32_t)(j * qbox * 128), tmap_q, bar, c * 64, row, pol);
     }
     bytes += (uint32_t)qbox * 128u;
   }
   return bytes;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+// Error path of the pair variant: copies a CTA issued complete on the leader's
+// barriers, which it cannot wait on, so it lets them land for a fixed time
+// (far above any copy's latency) before its shared memory may be released.
+__device__ __forceinline__ void settle_inflight_copies() {
+  const uint64_t t0 = global_timer_ns();
+  while (global_timer_ns() - t0 < 200000ull) __nanosleep(1000);
+}
+
+// kPair = false: 2-CTA clusters (S-CTA, O-CTA), one per 128-row group.
+// kPair = true: 4-CTA clusters (S pair, O pair), one per two row groups; every
+// tcgen05 instruction of this variant is a cta_group::2 one.
+// The cluster shape is set at launch (2 or 4 CTAs along x).
+template <bool kPair>
+__global__ void __launch_bounds__(kThreads, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_q,
-              const __grid_constant__ CUtensorMap tmap_v,
+              const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_kv2,
               const DecodeParams P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -238,12 +277,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
     if (tid == 0) atomicCAS(P.err, 0, kErrBadSmemAlign);
     return;
   }
-  const uint32_t rank = cluster_ctarank();
-  const int cluster_id = blockIdx.x >> 1;
-  const int groups = P.h_kv * P.n_rg;
+  constexpr int kClusterCtas = kPair ? 4 : 2;
+  const uint32_t crank = cluster_ctarank();
+  // role: 0 = S-CTA, 1 = O-CTA; half: which CTA of the pair (pair variant)
+  const uint32_t rank = kPair ? (crank >> 1) : crank;
+  const uint32_t half = kPair ? (crank & 1u) : 0u;
+  const bool leader = half == 0;
+  const uint32_t lead_rank = crank & ~1u;             // the pair's MMA-issuing CTA
+  const uint32_t mate = crank ^ 1u;                   // the other CTA of the pair
+  const uint16_t pair_mask = (uint16_t)(3u << lead_rank);
+  const int cluster_id = blockIdx.x / kClusterCtas;
+  const int units = kPair ? (P.n_rg + 1) / 2 : P.n_rg;  // clusters per KV head and part
+  const int groups = P.h_kv * units;
   const int part = cluster_id / groups;
-  const int g = (cluster_id % groups) / P.n_rg;
-  const int rg = (cluster_id % groups) % P.n_rg;
+  const int g = (cluster_id % groups) / units;
+  const int rg = kPair ? 2 * ((cluster_id % groups) % units) + (int)half : (cluster_id % groups) % units;
 
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + OFF_CTRL);
   SideSlot* side = reinterpret_cast<SideSlot*>(smem + OFF_SIDE);
@@ -254,12 +302,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
   if (tid == 0) {
     if (rank == 0) {
       for (int s = 0; s < kRing; ++s) {
-        mbar_init(bar(kBarRingFull + s), 2);  // one arrival per TMA producer
+        // one arrival per TMA producer; pair: the leader's producer arms both CTAs' bytes
+        mbar_init(bar(kBarRingFull + s), kPair ? 1 : 2);
         mbar_init(bar(kBarRingEmpty + s), 1);
       }
       for (int s = 0; s < 2; ++s) {
         mbar_init(bar(kBarSFull + s), 1);
-        mbar_init(bar(kBarSFree + s), 256);
+        mbar_init(bar(kBarSFree + s), kPair ? 2 : 256);  // pair: one arrival per S-CTA
       }
       mbar_init(bar(kBarQrFull), 1);
       mbar_init(bar(kBarQrEmpty), 1);
@@ -272,10 +321,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
       }
       for (int s = 0; s < kPSlots; ++s) {
         mbar_init(bar(kBarPFull + s), 1);
-        mbar_init(bar(kBarPCons + s), 1 + 8);
+        mbar_init(bar(kBarPCons + s), kPair ? 1 + 16 : 1 + 8);
+        mbar_init(bar(kBarPeerP + s), 1);
       }
       mbar_init(bar(kBarCmdFull), 1);
-      mbar_init(bar(kBarCmdDone), 256);
+      mbar_init(bar(kBarCmdDone), kPair ? 2 : 256);
     }
     mbar_init(bar(kBarDrain), 1);
     ctrl->abort_flag = 0;
@@ -286,13 +336,19 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
     }
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&ctrl->tmem_base), 512);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(smem_u32(&ctrl->tmem_base), 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(&ctrl->tmem_base), 512);
+      tmem_relinquish();
+    }
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmap_kv);
     tma_prefetch_desc(&tmap_q);
     tma_prefetch_desc(&tmap_v);
+    if (kPair) tma_prefetch_desc(&tmap_kv2);
   }
   tc_fence_before();
   __syncthreads();
@@ -309,11 +365,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
   // completion signals of the pieces it merges)
   if (tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const PartIter it(P, part);
-  const uint32_t peer = rank ^ 1u;
+  // the CTA on the other side of the P hand-off (S-CTA <-> O-CTA of a row group)
+  const uint32_t peer = kPair ? (crank ^ 2u) : (crank ^ 1u);
 
   if (rank == 0) {
     // =========================================================== S-CTA
     if ((warp == 0 || warp == 2) && lane == 0) {
+      if constexpr (!kPair) {
       // ---- two TMA producers walk the same chunk-stage sequence; every stage's
       // full barrier takes one arrival from each.  Producer 0 loads the query
       // chunks and page A of each pair, producer 1 page B: one thread alone
@@ -384,7 +442,65 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
           if (issued[s]) mbar_wait_drain(bar(kBarRingFull + s), issued_phase[s]);
         if (qr_issued) mbar_wait_drain(bar(kBarQrFull), qr_issued_phase);
       }
+      } else {
+        // ---- pair: the two producers of each S-CTA take turns over the stages.
+        // Each CTA loads its own row group's query and its own page of every
+        // pair (rank 0 page A, rank 1 page B; a missing page B reads as zeros,
+        // from outside the tensor map), the page in stages of two 64-column
+        // chunks; all bytes complete on the leader's barriers, which the
+        // leader's producer arms for both CTAs.
+        const int prod = warp >> 1;
+        Ring st;
+        uint32_t turn = 0;  // running stage count: stage k belongs to producer k % 2
+        uint32_t qr_phase = 0;
+        bool ok = true;
+        const uint64_t pol_q = policy_evict_last();
+        const uint64_t pol_kv = policy_evict_normal();
+        const uint32_t lead_full0 = map_to_rank(bar(kBarRingFull), lead_rank);
+        const uint32_t lead_qr = map_to_rank(bar(kBarQrFull), lead_rank);
+        const uint32_t q_bytes = load_q_chunk(P, &tmap_q, 0, 0, 0, g, rg, 0, 0, false) +
+                                 load_q_chunk(P, &tmap_q, 0, 0, 0, g, rg ^ 1, 0, 0, false);
+        for_each_piece(P, it, [&](int b, int p0, int p1, int) {
+          for (int c = 0; c < 8; ++c, ++turn) {
+            if ((turn & 1u) == (uint32_t)prod) {
+              ok = mbar_wait<true>(bar(kBarRingEmpty + st.idx), st.phase ^ 1u, abortf, P.err, kErrWaitBase + 1);
+              if (!ok) return false;
+              if (leader) mbar_arrive_expect_tx(bar(kBarRingFull + st.idx), q_bytes);
+              load_q_chunk<true>(P, &tmap_q, sbase + OFF_RING + st.idx * kChunkBytes, lead_full0 + 8u * st.idx,
+                                 b, g, rg, c, pol_q, true);
+            }
+            st.next(kRing);
+          }
+          if (prod == 0) {
+            ok = mbar_wait<true>(bar(kBarQrEmpty), qr_phase ^ 1u, abortf, P.err, kErrWaitBase + 2);
+            if (!ok) return false;
+            if (leader) mbar_arrive_expect_tx(bar(kBarQrFull), q_bytes);
+            load_q_chunk<true>(P, &tmap_q, sbase + OFF_QROPE, lead_qr, b, g, rg, 8, pol_q, true);
+            qr_phase ^= 1u;
+          }
+          for (int pa = p0; pa < p1; pa += 2) {
+            const int page = half == 0 ? load_page(P, b, pa) : (pa + 1 < p1 ? load_page(P, b, pa + 1) : P.num_pages);
+            for (int s = 0; s < 5; ++s, ++turn) {
+              if ((turn & 1u) == (uint32_t)prod) {
+                ok = mbar_wait<true>(bar(kBarRingEmpty + st.idx), st.phase ^ 1u, abortf, P.err, kErrWaitBase + 3);
+                if (!ok) return false;
+                const uint32_t dst = sbase + OFF_RING + st.idx * kChunkBytes;
+                const uint32_t fb = lead_full0 + 8u * st.idx;
+                if (leader) mbar_arrive_expect_tx(bar(kBarRingFull + st.idx), (s < 4 ? 4u : 2u) * kPageChunkBytes);
+                if (s < 4)  // chunks 2s and 2s+1 of the page, chunk-major
+                  tma_load_4d_pair(dst, &tmap_kv2, fb, 0, page * kPage, 2 * s, g, pol_kv);
+                else        // the RoPE chunk
+                  tma_load_3d_pair(dst, &tmap_kv, fb, 8 * 64, g, page * kPage, pol_kv);
+              }
+              st.next(kRing);
+            }
+          }
+          return true;
+        });
+        if (!ok) settle_inflight_copies();
+      }
     } else if (warp == 1 && lane == 0) {
+      if constexpr (!kPair) {
       // ---- MMA issuer: S = Q K^T for page pairs (N = 128) or a single page (N = 64)
       Ring st, sb;
       uint32_t qr_phase = 0;
@@ -463,6 +579,79 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
       });
       tc_commit(bar(kBarDrain));
       mbar_wait_drain(bar(kBarDrain), 0);
+      } else if (leader) {
+        // ---- pair MMA issuer (rank 0): S = Q K^T of both row groups, M = 256
+        // (rows of rank 0 then rank 1), N = 128 (page A from rank 0's shared
+        // memory, page B from rank 1's), K in stages of two chunks
+        Ring st, sb;
+        uint32_t qr_phase = 0;
+        const uint32_t idesc = make_idesc_bf16(256, 128, 0, 0);
+        const uint64_t ring_desc0 = make_smem_desc(sbase + OFF_RING, 16, 1024, 2);
+        const uint64_t qr_desc = make_smem_desc(sbase + OFF_QROPE, 16, 1024, 2);
+        const uint32_t ring_empty0 = bar(kBarRingEmpty);
+        const uint32_t ring_full0 = bar(kBarRingFull);
+        for_each_piece(P, it, [&](int, int p0, int p1, int) {
+          // each CTA's latent query chunks into its own TMEM columns [32c, 32c + 32)
+          for (int c = 0; c < 8; ++c) {
+            if (!mbar_wait<true>(ring_full0 + 8u * st.idx, st.phase, abortf, P.err, kErrWaitBase + 9))
+              return false;
+            tc_fence_after();
+            const uint64_t qd = ring_desc0 + (uint64_t)(st.idx * (kChunkBytes >> 4));
+#pragma unroll
+            for (int k = 0; k < 4; ++k) tmem_cp_128x256b_pair(tmem + kTmemQ + 32u * c + 8u * k, qd + 2 * k);
+            tc_commit_pair_mc(ring_empty0 + 8u * st.idx, pair_mask);
+            st.next(kRing);
+          }
+          bool first = true;
+          for (int pa = p0; pa < p1; pa += 2) {
+            const bool last_pair = pa + 2 >= p1;
+            if (!mbar_wait<true>(bar(kBarSFree + sb.idx), sb.phase ^ 1u, abortf, P.err, kErrWaitBase + 4))
+              return false;
+            const uint32_t dS = tmem + kTmemS + 128u * sb.idx;
+            for (int s = 0; s < 4; ++s) {
+              if (!mbar_wait<true>(ring_full0 + 8u * st.idx, st.phase, abortf, P.err, kErrWaitBase + 6))
+                return false;
+              tc_fence_after();
+              const uint64_t bd = ring_desc0 + (uint64_t)(st.idx * (kChunkBytes >> 4));
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                const int c = 2 * s + j;
+                const uint32_t a = tmem + kTmemQ + 32u * c;
+                const uint64_t bj = bd + (uint64_t)(j * (kPageChunkBytes >> 4));
+                mma_ts_pair(dS, a, bj, idesc, c > 0);
+                mma_ts_pair(dS, a + 8, bj + 2, idesc, 1);
+                mma_ts_pair(dS, a + 16, bj + 4, idesc, 1);
+                mma_ts_pair(dS, a + 24, bj + 6, idesc, 1);
+              }
+              tc_commit_pair_mc(ring_empty0 + 8u * st.idx, pair_mask);
+              st.next(kRing);
+            }
+            if (!mbar_wait<true>(ring_full0 + 8u * st.idx, st.phase, abortf, P.err, kErrWaitBase + 7))
+              return false;
+            if (first) {
+              if (!mbar_wait<true>(bar(kBarQrFull), qr_phase, abortf, P.err, kErrWaitBase + 8)) return false;
+              qr_phase ^= 1u;
+            }
+            tc_fence_after();
+            {
+              const uint64_t bd = ring_desc0 + (uint64_t)(st.idx * (kChunkBytes >> 4));
+              mma_ss_pair(dS, qr_desc, bd, idesc, 1);
+              mma_ss_pair(dS, qr_desc + 2, bd + 2, idesc, 1);
+              mma_ss_pair(dS, qr_desc + 4, bd + 4, idesc, 1);
+              mma_ss_pair(dS, qr_desc + 6, bd + 6, idesc, 1);
+              tc_commit_pair_mc(ring_empty0 + 8u * st.idx, pair_mask);
+              st.next(kRing);
+            }
+            tc_commit_pair_mc(bar(kBarSFull + sb.idx), pair_mask);
+            if (last_pair) tc_commit_pair_mc(bar(kBarQrEmpty), pair_mask);
+            sb.next(2);
+            first = false;
+          }
+          return true;
+        });
+        tc_commit_pair(bar(kBarDrain));
+        mbar_wait_drain(bar(kBarDrain), 0);
+      }
     } else if (warp >= 4) {
       // ---- two softmax warpgroups: thread (wg, r) owns query row r; of each page
       // pair, warpgroup 0 handles the first page and warpgroup 1 the second
@@ -498,8 +687,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
           const int npg = (pa + 1 < p1) ? 2 : 1;
           const bool last_pair = pa + 2 >= p1;
           const bool mine = wg < npg;  // uniform per group
-          ok = named_bar_and(bar_all, 256, mbar_wait(bar(kBarSFull + sb.idx), sb.phase, abortf, P.err,
-                                                     kErrWaitBase + 10));
+          ok = named_bar_and(bar_all, 256, mbar_wait<kPair>(bar(kBarSFull + sb.idx), sb.phase, abortf, P.err,
+                                                            kErrWaitBase + 10));
           if (!ok) return false;
           tc_fence_after();
           const int jw = (pa + wg) * kPage;  // first token of this group's page
@@ -511,7 +700,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
             for (int j = 0; j < 32; ++j) { s0[j] = 0xff800000u; s1[j] = 0xff800000u; }  // -inf
           }
           tc_fence_before();
-          mbar_arrive(bar(kBarSFree + sb.idx));
+          const uint32_t s_used = sb.idx;
+          if constexpr (!kPair) mbar_arrive(bar(kBarSFree + s_used));
           sb.next(2);
           const bool tail = mine && (jw + kPage - 1 > limit);
           if (tail) {
@@ -536,6 +726,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
           float* xm = xmax + (npair & 1u) * (2 * kRows);
           xm[wg * kRows + r] = mloc;
           named_bar_sync(bar_all, 256);
+          if constexpr (kPair) {
+            // all 256 threads have read this CTA's S tile: one arrival per CTA on
+            // the leader's barrier releases it for the next pair's MMAs
+            if (tid == 128) {
+              if (leader)
+                mbar_arrive(bar(kBarSFree + s_used));
+              else
+                mbar_arrive_remote(map_to_rank(bar(kBarSFree + s_used), lead_rank));
+            }
+          }
           const float mx = fmaxf(mloc, xm[(wg ^ 1) * kRows + r]);
           // identical lazy-rescale update in both groups
           const float mxs = (mx == -INFINITY) ? -INFINITY : mx * c;
@@ -622,7 +822,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
             if (pslot >= 0) {  // split piece: signal the merge kernel (lse half)
               __threadfence();
               named_bar_sync(bar_wg, 128);
-              if (r == 0) atomicAdd(&P.seq_done[((size_t)b * P.h_kv + g) * P.n_rg + rg], 1);
+              if (r == 0 && rg < P.n_rg) atomicAdd(&P.seq_done[((size_t)b * P.h_kv + g) * P.n_rg + rg], 1);
             }
           }
         }
@@ -632,6 +832,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
   } else {
     // =========================================================== O-CTA
     if (warp == 0 && lane == 0) {
+      if constexpr (!kPair) {
       // ---- TMA producer: value part of each page as two half-page stages
       Ring st;
       bool ok = true;
@@ -660,7 +861,33 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
         for (int s = 0; s < kVStages; ++s)
           if (issued[s]) mbar_wait_drain(bar(kBarVFull + s), issued_phase[s]);
       }
+      } else {
+        // ---- pair: this CTA's half of each page's value columns, chunks
+        // {2h, 2h+1} for the first N = 256 MMA and {4+2h, 5+2h} for the second
+        // (h = this CTA's half), one 32 KB stage per page, completing on the
+        // leader's barrier (armed there for both CTAs)
+        Ring st;
+        bool ok = true;
+        const uint64_t pol = policy_evict_first();
+        const uint32_t lead_vfull0 = map_to_rank(bar(kBarVFull), lead_rank);
+        for_each_piece(P, it, [&](int b, int p0, int p1, int) {
+          for (int p = p0; p < p1; ++p) {
+            const int page = load_page(P, b, p);
+            ok = mbar_wait<true>(bar(kBarVEmpty + st.idx), st.phase ^ 1u, abortf, P.err, kErrWaitBase + 12);
+            if (!ok) return false;
+            if (leader) mbar_arrive_expect_tx(bar(kBarVFull + st.idx), 2 * kVStageBytes);
+            const uint32_t dst = sbase + OFF_V + st.idx * kVStageBytes;
+            const uint32_t fb = lead_vfull0 + 8u * st.idx;
+            tma_load_4d_pair(dst, &tmap_kv2, fb, 0, page * kPage, 2 * (int)half, g, pol);
+            tma_load_4d_pair(dst + 2 * kPageChunkBytes, &tmap_kv2, fb, 0, page * kPage, 4 + 2 * (int)half, g, pol);
+            st.next(kVStages);
+          }
+          return true;
+        });
+        if (!ok) settle_inflight_copies();
+      }
     } else if (warp == 1 && lane == 0) {
+      if constexpr (!kPair) {
       // ---- MMA issuer: O += P V, plus the command stream to the correction warps
       Ring st;
       uint32_t kp = 0, done_phase = 0, drain_phase = 0;
@@ -735,6 +962,93 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
       if (pending_epilogue) mbar_wait(bar(kBarCmdDone), done_phase, abortf, nullptr, 0);
       tc_commit(bar(kBarDrain));
       mbar_wait_drain(bar(kBarDrain), drain_phase);
+      } else if (leader) {
+        // ---- pair MMA issuer (rank 2): O += P V for both row groups, M = 256
+        // (P rows of rank 2 then rank 3), N = 256 twice (value columns split
+        // between the two CTAs), plus the command stream to both CTAs'
+        // correction warps
+        Ring st;
+        uint32_t kp = 0, done_phase = 0, drain_phase = 0;
+        bool pending_epilogue = false, ok = true;
+        const uint32_t idesc = make_idesc_bf16(256, 256, 0, 1);
+        const uint64_t v_desc0 = make_smem_desc(sbase + OFF_V, 8192, 1024, 2);
+        const uint64_t p_desc0 = make_smem_desc(sbase + OFF_P, 16, 1024, 2);
+        const uint32_t mate_side = map_to_rank(smem_u32(side), mate);
+        const uint32_t mate_mail = map_to_rank(smem_u32(mail), mate);
+        const uint32_t mate_cmdfull = map_to_rank(bar(kBarCmdFull), mate);
+        auto post = [&](int cmd, int slot, int b, int pslot) {
+          mail->cmd = cmd;
+          mail->slot = slot;
+          mail->b = b;
+          mail->part_slot = pslot;
+          st_cluster_u32(mate_mail + (uint32_t)offsetof(Mailbox, cmd), (uint32_t)cmd);
+          st_cluster_u32(mate_mail + (uint32_t)offsetof(Mailbox, slot), (uint32_t)slot);
+          st_cluster_u32(mate_mail + (uint32_t)offsetof(Mailbox, b), (uint32_t)b);
+          st_cluster_u32(mate_mail + (uint32_t)offsetof(Mailbox, part_slot), (uint32_t)pslot);
+          tc_fence_before();
+          mbar_arrive(bar(kBarCmdFull));
+          mbar_arrive_remote(mate_cmdfull);
+        };
+        for_each_piece(P, it, [&](int b, int p0, int p1, int ordinal) {
+          for (int p = p0; p < p1; ++p, ++kp) {
+            const uint32_t ps = kp % kPSlots, pph = (kp / kPSlots) & 1u;
+            if (!mbar_wait<true>(bar(kBarPFull + ps), pph, abortf, P.err, kErrWaitBase + 13)) return false;
+            if (!mbar_wait<true>(bar(kBarPeerP + ps), pph, abortf, P.err, kErrWaitBase + 24)) return false;
+            const volatile uint32_t* wf = side[ps].wflag;
+            const uint32_t ms = mate_side + ps * kSideBytes;  // wflag[0..3] lead the side slot
+            const bool resc = ((wf[0] | wf[1] | wf[2] | wf[3]) | (ld_cluster_u32(ms) | ld_cluster_u32(ms + 4) |
+                                                                 ld_cluster_u32(ms + 8) | ld_cluster_u32(ms + 12))) != 0u;
+            const bool first = (p == p0), last = (p == p1 - 1);
+            if (first && pending_epilogue) {  // accumulators still being drained by the epilogue
+              ok = mbar_wait<true>(bar(kBarCmdDone), done_phase, abortf, P.err, kErrWaitBase + 14);
+              done_phase ^= 1u;
+              pending_epilogue = false;
+              if (!ok) return false;
+            }
+            if (resc && !first) {
+              // a row's reference max moved in either row group: finish all issued
+              // MMAs, then both CTAs rescale their O rows
+              tc_commit_pair(bar(kBarDrain));
+              ok = mbar_wait(bar(kBarDrain), drain_phase, abortf, P.err, kErrWaitBase + 15);
+              drain_phase ^= 1u;
+              if (!ok) return false;
+              post(kCmdRescale, (int)ps, 0, 0);
+              ok = mbar_wait<true>(bar(kBarCmdDone), done_phase, abortf, P.err, kErrWaitBase + 16);
+              done_phase ^= 1u;
+              if (!ok) return false;
+            }
+            if (!mbar_wait<true>(bar(kBarVFull + st.idx), st.phase, abortf, P.err, kErrWaitBase + 17))
+              return false;
+            tc_fence_after();
+            const uint64_t pd = p_desc0 + (uint64_t)(ps * (kPBytes >> 4));
+            const uint64_t vd = v_desc0 + (uint64_t)(st.idx * (kVStageBytes >> 4));
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+              const uint64_t vn = vd + (uint64_t)(n * (2 * kPageChunkBytes >> 4));
+              const uint32_t d = tmem + kTmemO + 256u * n;
+              mma_ss_pair(d, pd, vn, idesc, !first);
+              mma_ss_pair(d, pd + 2, vn + 128, idesc, 1);
+              mma_ss_pair(d, pd + 4, vn + 256, idesc, 1);
+              mma_ss_pair(d, pd + 6, vn + 384, idesc, 1);
+            }
+            tc_commit_pair_mc(bar(kBarVEmpty + st.idx), pair_mask);
+            st.next(kVStages);
+            tc_commit_pair_mc(bar(kBarPCons + ps), pair_mask);  // P slots consumed -> relay warps
+            if (last) {
+              tc_commit_pair(bar(kBarDrain));
+              ok = mbar_wait(bar(kBarDrain), drain_phase, abortf, P.err, kErrWaitBase + 18);
+              drain_phase ^= 1u;
+              if (!ok) return false;
+              post(kCmdEpilogue, 0, b, piece_slot(P, b, ordinal));
+              pending_epilogue = true;
+            }
+          }
+          return true;
+        });
+        if (pending_epilogue) mbar_wait<true>(bar(kBarCmdDone), done_phase, abortf, nullptr, 0);
+        tc_commit_pair(bar(kBarDrain));
+        mbar_wait_drain(bar(kBarDrain), drain_phase);
+      }
     } else if (warp == 2 && lane == 0) {
       // ---- relay: re-arm a consumed P slot and hand it back to the S-CTA
       uint32_t kp = 0;
@@ -742,7 +1056,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
       for_each_piece(P, it, [&](int, int p0, int p1, int) {
         for (int p = p0; p < p1; ++p, ++kp) {
           const uint32_t ps = kp % kPSlots, pph = (kp / kPSlots) & 1u;
-          if (!mbar_wait(bar(kBarPCons + ps), pph, abortf, P.err, kErrWaitBase + 19)) return false;
+          if (!mbar_wait<kPair>(bar(kBarPCons + ps), pph, abortf, P.err, kErrWaitBase + 19)) return false;
           mbar_arrive_expect_tx(bar(kBarPFull + ps), kPFullTx);
           mbar_arrive_remote(pfree_remote + ps * 8u);
         }
@@ -759,6 +1073,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
                                kErrWaitBase + 22))
             return false;
           mbar_arrive_remote(sfree_remote + (kp % kStageBufs) * 8u);
+          if constexpr (kPair) mbar_arrive_remote(map_to_rank(bar(kBarPeerP + kp % kPSlots), mate));
         }
         return true;
       });
@@ -781,12 +1096,29 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
       auto agree = [&](bool ok) { return named_bar_and(4, 256, ok); };
       // one command from the MMA thread
       auto wait_cmd = [&]() {
-        if (!agree(mbar_wait(bar(kBarCmdFull), cmd_phase, abortf, P.err, kErrWaitBase + 20)))
+        if (!agree(mbar_wait<kPair>(bar(kBarCmdFull), cmd_phase, abortf, P.err, kErrWaitBase + 20)))
           return false;
         cmd_phase ^= 1u;
         tc_fence_after();
         return true;
       };
+      // a command is done: every thread arrives (single CTA), or, in the pair
+      // variant, one arrival per CTA on the leader's barrier once all 256 are done
+      auto cmd_done = [&]() {
+        tc_fence_before();
+        if constexpr (kPair) {
+          named_bar_sync(4, 256);
+          if (tid == 128) {
+            if (leader)
+              mbar_arrive(bar(kBarCmdDone));
+            else
+              mbar_arrive_remote(map_to_rank(bar(kBarCmdDone), lead_rank));
+          }
+        } else {
+          mbar_arrive(bar(kBarCmdDone));
+        }
+      };
+      const uint32_t mate_side = kPair ? map_to_rank(smem_u32(side), mate) : 0u;
       for_each_piece(P, it, [&](int, int p0, int p1, int) {
         // lr: this group's half of the row's sum of the bf16 weights the MMA
         // multiplies, rescaled with O
@@ -796,7 +1128,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
           if (!agree(mbar_wait<true>(bar(kBarPFull + ps), pph, abortf, P.err, kErrWaitBase + 23)))
             return false;
           const volatile uint32_t* wf = side[ps].wflag;
-          const bool resc = p != p0 && (wf[0] | wf[1] | wf[2] | wf[3]) != 0u;
+          uint32_t any = wf[0] | wf[1] | wf[2] | wf[3];
+          if constexpr (kPair) {
+            // the MMA thread rescales when either row group moved a reference max:
+            // read the mate's flags once its P slot has landed
+            if (!agree(mbar_wait<true>(bar(kBarPeerP + ps), pph, abortf, P.err, kErrWaitBase + 25)))
+              return false;
+            const uint32_t ms = mate_side + ps * kSideBytes;
+            any |= ld_cluster_u32(ms) | ld_cluster_u32(ms + 4) | ld_cluster_u32(ms + 8) | ld_cluster_u32(ms + 12);
+          }
+          const bool resc = p != p0 && any != 0u;
           const float a = side[ps].alpha[r];
           const uint8_t* prow = smem + OFF_P + ps * kPBytes + prow_off;
           float s4[4];
@@ -810,7 +1151,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
           }
           lr = fmaf(lr, a, (s4[0] + s4[1]) + (s4[2] + s4[3]));
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(kBarPCons + ps));  // this warp is done with the slot
+          if (lane == 0) {
+            mbar_arrive(bar(kBarPCons + ps));  // this warp is done with the slot
+            // pair: and with the mate's flags, so the mate's slot may be refilled
+            if constexpr (kPair) mbar_arrive_remote(map_to_rank(bar(kBarPCons + ps), mate));
+          }
           if (resc) {
             // the MMA thread drains and posts a rescale before this page's MMAs
             if (!wait_cmd()) return false;
@@ -825,12 +1170,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
               }
               tmem_wait_st();
             }
-            tc_fence_before();
-            mbar_arrive(bar(kBarCmdDone));
+            cmd_done();
           }
         }
         {
-          const bool okc = mbar_wait(bar(kBarCmdFull), cmd_phase, abortf, P.err, kErrWaitBase + 20);
+          const bool okc = mbar_wait<kPair>(bar(kBarCmdFull), cmd_phase, abortf, P.err, kErrWaitBase + 20);
           float* xr = mail->lr_x[npiece & 1u][0];
           xr[wg * kRows + r] = lr;  // exchanged with the other group at the barrier
           if (!agree(okc)) return false;  // the piece's epilogue command
@@ -893,10 +1237,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
             // signal the merge kernel (partial o half) once all 256 threads stored
             __threadfence();
             named_bar_sync(4, 256);
-            if (tid == 128) atomicAdd(&P.seq_done[((size_t)b * P.h_kv + g) * P.n_rg + rg], 1);
+            if (tid == 128 && rg < P.n_rg) atomicAdd(&P.seq_done[((size_t)b * P.h_kv + g) * P.n_rg + rg], 1);
           }
-          tc_fence_before();
-          mbar_arrive(bar(kBarCmdDone));
+          cmd_done();
           return true;
         }
       });
@@ -911,7 +1254,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
   cluster_wait();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    if constexpr (kPair)
+      tmem_dealloc_pair(tmem, 512);
+    else
+      tmem_dealloc(tmem, 512);
   }
 }
 
@@ -923,46 +1269,58 @@ cudaError_t decode_prepare(int device) {
   static bool done[64] = {};
   if (device >= 0 && device < 64 && done[device]) return cudaSuccess;
   cudaError_t e =
-      cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+      cudaFuncSetAttribute(decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e == cudaSuccess && device >= 0 && device < 64) done[device] = true;
   return e;
 }
 
-int decode_max_active_clusters(int device, int* out) {
+int decode_max_active_clusters(int device, bool pair, int* out) {
   cudaError_t e = decode_prepare(device);
   if (e != cudaSuccess) return (int)e;
+  const int ctas = pair ? 4 : 2;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * 512, 1, 1);
+  cfg.gridDim = dim3(ctas * 512, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.x = ctas;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  e = cudaOccupancyMaxActiveClusters(&n, decode_kernel, &cfg);
+  e = pair ? cudaOccupancyMaxActiveClusters(&n, decode_kernel<true>, &cfg)
+           : cudaOccupancyMaxActiveClusters(&n, decode_kernel<false>, &cfg);
   if (e != cudaSuccess) return (int)e;
   *out = n;
   return 0;
 }
 
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, const CUtensorMap& tmap_q,
-                          const CUtensorMap& tmap_v, cudaStream_t stream) {
-  const int clusters = p.num_parts * p.h_kv * p.n_rg;
+                          const CUtensorMap& tmap_v, const CUtensorMap& tmap_kv2, bool pair,
+                          cudaStream_t stream) {
+  const int ctas = pair ? 4 : 2;
+  const int units = pair ? (p.n_rg + 1) / 2 : p.n_rg;
+  const int clusters = p.num_parts * p.h_kv * units;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.gridDim = dim3(ctas * clusters, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = ctas;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel, tmap_kv, tmap_q, tmap_v, p);
+  cfg.numAttrs = 2;
+  return pair ? cudaLaunchKernelEx(&cfg, decode_kernel<true>, tmap_kv, tmap_q, tmap_v, tmap_kv2, p)
+              : cudaLaunchKernelEx(&cfg, decode_kernel<false>, tmap_kv, tmap_q, tmap_v, tmap_kv2, p);
 }
 
 }  // namespace pmla

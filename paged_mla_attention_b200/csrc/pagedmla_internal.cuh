@@ -94,9 +94,14 @@ WorkspaceLayout workspace_layout(int batch, int R, int h_kv, int num_parts);
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* meta,
                             int32_t* num_splits, cudaStream_t stream);
 cudaError_t decode_prepare(int device);  // one-time per-device kernel attributes
-int decode_max_active_clusters(int device, int* out);
+// Clusters of the decode kernel resident at once: 2-CTA clusters (pair = false,
+// one per 128-row group) or 4-CTA clusters (pair = true, one per two row groups).
+int decode_max_active_clusters(int device, bool pair, int* out);
+// The 4-CTA variant is used when a KV head has two or more row groups.
+inline bool decode_uses_pairs(int n_rg) { return n_rg >= 2; }
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, const CUtensorMap& tmap_q,
-                          const CUtensorMap& tmap_v, cudaStream_t stream);
+                          const CUtensorMap& tmap_v, const CUtensorMap& tmap_kv2, bool pair,
+                          cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 cudaError_t launch_clear_counters(int* ctr, int n, cudaStream_t stream);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);

@@ -133,6 +133,32 @@ def test_lazy_rescale_path():
     _check(inp, "rescale")
 
 
+def test_pair_clusters_rescale_one_row_group():
+    # s_q = 2, causal, 128 heads: both row groups (query token 0, query token 1)
+    # share one 4-CTA cluster.  The last cached token scores far above all others
+    # and only query token 1 sees it, so only the second row group moves its
+    # reference max there: the O pair must rescale on the other CTA's flag too.
+    L = 64 * 12 + 7
+    inp = _small([L, 300], s_q=2, h_q=128, causal=True, seed=35)
+    kv = W.bf16_bits_to_f32(inp["kvcache"]).copy()
+    q = W.bf16_bits_to_f32(inp["q"]).copy()
+    last = inp["block_table"][0][(L - 1) // 64]
+    kv[last, (L - 1) % 64, 0, 570] = 200.0     # a RoPE column: not part of the values
+    q[..., 570] = np.abs(q[..., 570]) + 0.5
+    t = np.arange(L - 1)
+    pages = inp["block_table"][0][t // 64]
+    kv[pages, t % 64, 0, 570] = np.linspace(-4.0, 4.0, L - 1)   # a climbing max for both groups
+    inp["kvcache"] = W.f32_to_bf16_bits(kv)
+    inp["q"] = W.f32_to_bf16_bits(q)
+    _check(inp, "pair rescale")
+
+
+def test_pair_clusters_odd_row_groups():
+    # s_q = 3 x 128 heads: three row groups, so the second 4-CTA cluster's upper
+    # half has no rows at all
+    _check(_small([5, 200, 1300, 64], s_q=3, h_q=128, causal=True, seed=36), "R=384")
+
+
 @pytest.mark.parametrize("seed", range(6))
 def test_scheduler_invariants(seed):
     import torch
