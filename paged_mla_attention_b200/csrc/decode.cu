@@ -114,7 +114,9 @@ enum : int {
   kBarPFull = kBarVEmpty + kVStages,     // O [kPSlots] P slot written (armed + bulk-copy tx)
   kBarPCons = kBarPFull + kPSlots,       // O [kPSlots] P slot consumed (commit + 8 warps; pair: + 8 of the mate)
   kBarPeerP = kBarPCons + kPSlots,       // O [kPSlots] pair: the mate O-CTA's P slot landed (remote arrival)
-  kBarCmdFull = kBarPeerP + kPSlots,     // O mailbox command posted (1)
+  kBarFlagsRead = kBarPeerP + kPSlots,   // O [kPSlots] pair: this CTA's 8 correction warps read the mate's flags
+  kBarSFreeFwd = kBarFlagsRead + kPSlots,  // S [2] pair, odd CTA: its softmax read S (relayed to the leader)
+  kBarCmdFull = kBarSFreeFwd + 2,        // O mailbox command posted (1)
   kBarCmdDone = kBarCmdFull + 1,         // O command done (256; pair: 1 per O-CTA, on rank 2)
   kBarDrain = kBarCmdDone + 1,           // both: all issued MMAs complete
   kNumBars = kBarDrain + 1
@@ -312,6 +314,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
       }
       mbar_init(bar(kBarQrFull), 1);
       mbar_init(bar(kBarQrEmpty), 1);
+      for (int s = 0; s < 2; ++s) mbar_init(bar(kBarSFreeFwd + s), 1);
       for (int s = 0; s < kPSlots; ++s) mbar_init(bar(kBarPFree + s), 1);
       for (int s = 0; s < kStageBufs; ++s) mbar_init(bar(kBarStageFree + s), 1);
     } else {
@@ -321,8 +324,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
       }
       for (int s = 0; s < kPSlots; ++s) {
         mbar_init(bar(kBarPFull + s), 1);
-        mbar_init(bar(kBarPCons + s), kPair ? 1 + 16 : 1 + 8);
+        // commit + this CTA's 8 correction warps (+ pair: the mate's, relayed once)
+        mbar_init(bar(kBarPCons + s), kPair ? 1 + 8 + 1 : 1 + 8);
         mbar_init(bar(kBarPeerP + s), 1);
+        mbar_init(bar(kBarFlagsRead + s), 8);
       }
       mbar_init(bar(kBarCmdFull), 1);
       mbar_init(bar(kBarCmdDone), kPair ? 2 : 256);
@@ -608,11 +613,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
             if (!mbar_wait<true>(bar(kBarSFree + sb.idx), sb.phase ^ 1u, abortf, P.err, kErrWaitBase + 4))
               return false;
             const uint32_t dS = tmem + kTmemS + 128u * sb.idx;
+            // the pair's five stages (four of two chunks, then the RoPE chunk), issued
+            // unrolled with precomputed stage indices: the per-stage waits stay (TMA
+            // streams stage by stage) but no ring arithmetic or fence sits between MMAs
+            tc_fence_after();
+            uint32_t sidx[5], sph[5];
+#pragma unroll
+            for (int s = 0; s < 5; ++s) {
+              sidx[s] = st.idx;
+              sph[s] = st.phase;
+              st.next(kRing);
+            }
+#pragma unroll
             for (int s = 0; s < 4; ++s) {
-              if (!mbar_wait<true>(ring_full0 + 8u * st.idx, st.phase, abortf, P.err, kErrWaitBase + 6))
-                return false;
-              tc_fence_after();
-              const uint64_t bd = ring_desc0 + (uint64_t)(st.idx * (kChunkBytes >> 4));
+              if (!mbar_wait(ring_full0 + 8u * sidx[s], sph[s], abortf, P.err, kErrWaitBase + 6)) return false;
+              const uint64_t bd = ring_desc0 + (uint64_t)(sidx[s] * (kChunkBytes >> 4));
 #pragma unroll
               for (int j = 0; j < 2; ++j) {
                 const int c = 2 * s + j;
@@ -623,24 +638,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
                 mma_ts_pair(dS, a + 16, bj + 4, idesc, 1);
                 mma_ts_pair(dS, a + 24, bj + 6, idesc, 1);
               }
-              tc_commit_pair_mc(ring_empty0 + 8u * st.idx, pair_mask);
-              st.next(kRing);
+              tc_commit_pair_mc(ring_empty0 + 8u * sidx[s], pair_mask);
             }
-            if (!mbar_wait<true>(ring_full0 + 8u * st.idx, st.phase, abortf, P.err, kErrWaitBase + 7))
-              return false;
+            if (!mbar_wait(ring_full0 + 8u * sidx[4], sph[4], abortf, P.err, kErrWaitBase + 7)) return false;
             if (first) {
               if (!mbar_wait<true>(bar(kBarQrFull), qr_phase, abortf, P.err, kErrWaitBase + 8)) return false;
               qr_phase ^= 1u;
             }
-            tc_fence_after();
             {
-              const uint64_t bd = ring_desc0 + (uint64_t)(st.idx * (kChunkBytes >> 4));
+              const uint64_t bd = ring_desc0 + (uint64_t)(sidx[4] * (kChunkBytes >> 4));
               mma_ss_pair(dS, qr_desc, bd, idesc, 1);
               mma_ss_pair(dS, qr_desc + 2, bd + 2, idesc, 1);
               mma_ss_pair(dS, qr_desc + 4, bd + 4, idesc, 1);
               mma_ss_pair(dS, qr_desc + 6, bd + 6, idesc, 1);
-              tc_commit_pair_mc(ring_empty0 + 8u * st.idx, pair_mask);
-              st.next(kRing);
+              tc_commit_pair_mc(ring_empty0 + 8u * sidx[4], pair_mask);
             }
             tc_commit_pair_mc(bar(kBarSFull + sb.idx), pair_mask);
             if (last_pair) tc_commit_pair_mc(bar(kBarQrEmpty), pair_mask);
@@ -652,6 +663,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
         tc_commit_pair(bar(kBarDrain));
         mbar_wait_drain(bar(kBarDrain), 0);
       }
+    } else if (kPair && warp == 3 && lane == 0 && !leader) {
+      // ---- pair, odd S-CTA: forward "this CTA's S tile was read" to the leader
+      Ring sb;
+      const uint32_t lead_sfree = map_to_rank(bar(kBarSFree), lead_rank);
+      for_each_piece(P, it, [&](int, int p0, int p1, int) {
+        for (int pa = p0; pa < p1; pa += 2) {
+          if (!mbar_wait(bar(kBarSFreeFwd + sb.idx), sb.phase, abortf, P.err, kErrWaitBase + 26)) return false;
+          mbar_arrive_remote(lead_sfree + 8u * sb.idx);
+          sb.next(2);
+        }
+        return true;
+      });
     } else if (warp >= 4) {
       // ---- two softmax warpgroups: thread (wg, r) owns query row r; of each page
       // pair, warpgroup 0 handles the first page and warpgroup 1 the second
@@ -730,10 +753,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
             // all 256 threads have read this CTA's S tile: one arrival per CTA on
             // the leader's barrier releases it for the next pair's MMAs
             if (tid == 128) {
+              // the odd CTA's arrival is relayed by warp 3: an arrival on another
+              // CTA's barrier takes ~1 us from a thread with stores in flight
               if (leader)
                 mbar_arrive(bar(kBarSFree + s_used));
               else
-                mbar_arrive_remote(map_to_rank(bar(kBarSFree + s_used), lead_rank));
+                mbar_arrive(bar(kBarSFreeFwd + s_used));
             }
           }
           const float mx = fmaxf(mloc, xm[(wg ^ 1) * kRows + r]);
@@ -1017,7 +1042,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
               done_phase ^= 1u;
               if (!ok) return false;
             }
-            if (!mbar_wait<true>(bar(kBarVFull + st.idx), st.phase, abortf, P.err, kErrWaitBase + 17))
+            if (!mbar_wait(bar(kBarVFull + st.idx), st.phase, abortf, P.err, kErrWaitBase + 17))
               return false;
             tc_fence_after();
             const uint64_t pd = p_desc0 + (uint64_t)(ps * (kPBytes >> 4));
@@ -1053,12 +1078,19 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
       // ---- relay: re-arm a consumed P slot and hand it back to the S-CTA
       uint32_t kp = 0;
       const uint32_t pfree_remote = map_to_rank(bar(kBarPFree), peer);
+      const uint32_t mate_pcons = kPair ? map_to_rank(bar(kBarPCons), mate) : 0u;
       for_each_piece(P, it, [&](int, int p0, int p1, int) {
         for (int p = p0; p < p1; ++p, ++kp) {
           const uint32_t ps = kp % kPSlots, pph = (kp / kPSlots) & 1u;
+          if constexpr (kPair) {
+            // this CTA's correction warps have read the mate's flags of this
+            // page: the mate may refill its slot once its own consumers are done
+            if (!mbar_wait(bar(kBarFlagsRead + ps), pph, abortf, P.err, kErrWaitBase + 27)) return false;
+            mbar_arrive_remote_relaxed(mate_pcons + ps * 8u);
+          }
           if (!mbar_wait<kPair>(bar(kBarPCons + ps), pph, abortf, P.err, kErrWaitBase + 19)) return false;
           mbar_arrive_expect_tx(bar(kBarPFull + ps), kPFullTx);
-          mbar_arrive_remote(pfree_remote + ps * 8u);
+          mbar_arrive_remote_relaxed(pfree_remote + ps * 8u);
         }
         return true;
       });
@@ -1072,8 +1104,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
           if (!mbar_wait<true>(bar(kBarPFull + kp % kPSlots), (kp / kPSlots) & 1u, abortf, P.err,
                                kErrWaitBase + 22))
             return false;
-          mbar_arrive_remote(sfree_remote + (kp % kStageBufs) * 8u);
-          if constexpr (kPair) mbar_arrive_remote(map_to_rank(bar(kBarPeerP + kp % kPSlots), mate));
+          mbar_arrive_remote_relaxed(sfree_remote + (kp % kStageBufs) * 8u);
+          if constexpr (kPair) mbar_arrive_remote_relaxed(map_to_rank(bar(kBarPeerP + kp % kPSlots), mate));
         }
         return true;
       });
@@ -1153,8 +1185,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
           __syncwarp();
           if (lane == 0) {
             mbar_arrive(bar(kBarPCons + ps));  // this warp is done with the slot
-            // pair: and with the mate's flags, so the mate's slot may be refilled
-            if constexpr (kPair) mbar_arrive_remote(map_to_rank(bar(kBarPCons + ps), mate));
+            // pair: and with the mate's flags (relay warp 2 tells the mate)
+            if constexpr (kPair) mbar_arrive(bar(kBarFlagsRead + ps));
           }
           if (resc) {
             // the MMA thread drains and posts a rescale before this page's MMAs

@@ -80,6 +80,15 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
                : "memory");
 }
 
+// Relaxed arrival on a peer CTA's barrier: no release fence, so the arriving
+// thread does not wait for its earlier memory operations (a release arrival
+// from a thread with writes in flight was measured at ~1.3 us, a relaxed one
+// returns at once).  For signals that publish no data of the arriving thread:
+// "a buffer you filled has been consumed / has landed".
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
