@@ -47,8 +47,12 @@ constexpr int kChunks = kDV / 8;  // 64 chunks of 8 columns
 // are in flight together.  Few slices suit sequences cut into few pieces (less
 // repeated lse work, fewer blocks waiting); many slices suit a long sequence
 // cut into many pieces, whose merge would otherwise run on a handful of SMs.
-template <int kQuarters, int kPieceBatch>
-__global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombineParams P) {
+// kGroups groups of 8 warps share a block and take the pieces in turns, each
+// group keeping kPieceBatch pieces' loads in flight; their sums meet in shared
+// memory (a sequence cut into ~70 pieces otherwise spends ~9 serial rounds of
+// load latency in one block).
+template <int kQuarters, int kPieceBatch, int kGroups = 1>
+__global__ void __launch_bounds__(kMergeThreads * kGroups) combine_kernel(const CombineParams P) {
   constexpr int kQCols = kDV / kQuarters;
   constexpr int kQChunks = kChunks / kQuarters;
   constexpr int kCPW = kQChunks / 8;  // chunks per warp
@@ -58,7 +62,8 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombinePar
   __shared__ float row_lse[kMergeRows];
   const int b = blockIdx.z;
   const int g = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = wid & 7, grp = wid >> 3;  // chunk warp within the group, piece group
   const int r0 = (blockIdx.x / kQuarters) * kMergeRows;
   const int quarter = blockIdx.x % kQuarters;
   const int s0 = P.num_splits[b];
@@ -107,7 +112,7 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombinePar
   for (int k0 = 0; k0 < n; k0 += kMaxPieces) {
     const int nk = min(n - k0, kMaxPieces);
     __syncthreads();
-    for (int k = warp; k < nk; k += 8)
+    for (int k = wid; k < nk; k += 8 * kGroups)
       wsh[k][lane] = valid ? __ldcg(P.part_lse + ((size_t)(s0 + k0 + k) * P.h_kv + g) * P.R + rr)
                            : -INFINITY;
     __syncthreads();
@@ -122,7 +127,7 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombinePar
     }
   }
   const float total = (m == -INFINITY) ? -INFINITY : m + __logf(z);
-  if (warp == 0) row_lse[lane] = total;
+  if (wid == 0) row_lse[lane] = total;
 
   float acc[kCPW][8];
 #pragma unroll
@@ -135,7 +140,7 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombinePar
                          ((size_t)(quarter * kQChunks + warp) * P.R + rr) * 2;
     const size_t piece_stride = (size_t)P.h_kv * kChunks * P.R * 2;  // float4s between slots
     const size_t chunk8 = (size_t)8 * P.R * 2;                       // float4s between chunks c, c+8
-    for (int k0 = 0; k0 < n; k0 += kPieceBatch) {
+    for (int k0 = grp * kPieceBatch; k0 < n; k0 += kPieceBatch * kGroups) {
       float w[kPieceBatch];
       float4 x[kPieceBatch][kCPW], y[kPieceBatch][kCPW];
 #pragma unroll
@@ -172,8 +177,26 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombinePar
         }
     }
   }
+  if constexpr (kGroups > 1) {
+    // the other groups' sums join group 0's
+    __shared__ float red[kGroups - 1][8][kCPW][8][kMergeRows];
+    if (grp > 0)
+#pragma unroll
+      for (int i = 0; i < kCPW; ++i)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) red[grp - 1][warp][i][u][lane] = acc[i][u];
+    __syncthreads();
+    if (grp == 0)
+#pragma unroll
+      for (int q = 0; q < kGroups - 1; ++q)
+#pragma unroll
+        for (int i = 0; i < kCPW; ++i)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) acc[i][u] += red[q][warp][i][u][lane];
+  }
 #pragma unroll
   for (int i = 0; i < kCPW; ++i) {
+    if (grp > 0) break;
     uint32_t pk[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -186,7 +209,7 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombinePar
 
   // rows r0.. of (b, g): row rr is query token rr / hpk, head g*hpk + rr % hpk
   constexpr int kVec = kQCols * 2 / 16;  // 16-byte pieces per row of the quarter
-  for (int e = threadIdx.x; e < kMergeRows * kVec; e += kMergeThreads) {
+  for (int e = threadIdx.x; e < kMergeRows * kVec; e += kMergeThreads * kGroups) {
     const int row = e / kVec, c = e % kVec;
     const int r = r0 + row;
     if (r >= P.R) continue;
@@ -195,7 +218,7 @@ __global__ void __launch_bounds__(kMergeThreads) combine_kernel(const CombinePar
         reinterpret_cast<uint4*>(P.o + ((size_t)(b * P.s_q + qi) * P.h_q + head) * kDV + quarter * kQCols) + c;
     *dst = *reinterpret_cast<const uint4*>(&tile[row][c * 8]);
   }
-  if (warp == 0 && valid && quarter == 0) {
+  if (wid == 0 && valid && quarter == 0) {
     const int qi = rr / P.hpk, head = g * P.hpk + rr % P.hpk;
     P.lse[((size_t)b * P.h_q + head) * P.s_q + qi] = row_lse[lane];
   }
@@ -241,7 +264,7 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
   const bool many = p.num_parts >= 2 * p.batch;
   const int slices = many ? 8 : 1;
   cfg.gridDim = dim3(((p.R + kMergeRows - 1) / kMergeRows) * slices, p.h_kv, p.batch);
-  cfg.blockDim = dim3(kMergeThreads, 1, 1);
+  cfg.blockDim = dim3(many ? 2 * kMergeThreads : kMergeThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -249,7 +272,7 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return many ? cudaLaunchKernelEx(&cfg, combine_kernel<8, 8>, p)
+  return many ? cudaLaunchKernelEx(&cfg, combine_kernel<8, 8, 2>, p)
               : cudaLaunchKernelEx(&cfg, combine_kernel<1, 1>, p);
 }
 
