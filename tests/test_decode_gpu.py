@@ -153,6 +153,13 @@ def test_pair_clusters_rescale_one_row_group():
     _check(inp, "pair rescale")
 
 
+def test_pair_clusters_two_kv_heads_and_non_causal():
+    # two row groups per KV head with two KV heads (h_q 256, h_kv 2, s_q 2), and
+    # the non-causal two-token case at 128 heads: both run the 4-CTA variant
+    _check(_small([130, 2000, 64, 1], s_q=2, h_q=256, h_kv=2, causal=True, seed=37), "pair h_kv=2")
+    _check(_small([700, 5, 3100], s_q=2, h_q=128, causal=False, seed=38), "pair non-causal")
+
+
 def test_pair_clusters_odd_row_groups():
     # s_q = 3 x 128 heads: three row groups, so the second 4-CTA cluster's upper
     # half has no rows at all
