@@ -296,6 +296,11 @@ PMLA_API int pmla_page_pool_release_sequence(pmla_page_pool* pool, const int32_t
  *   q_nope [tokens][heads][128], q_rope [tokens][heads][64], q_out [tokens][heads][576]
  *   o_latent [tokens][heads][512], o_out [tokens][heads][128]
  * Inputs 16-byte aligned, outputs 32-byte aligned, all device memory.
+ * Each runs as one kernel launched as a programmatic dependent of the kernel
+ * before it on `stream`: it may start, and prefetch the weight matrix into L2,
+ * before that kernel has completed; it reads nothing into the computation and
+ * writes nothing until that kernel has completed, so stream order holds as for
+ * a plain launch.
  * Errors: INVALID_ARG, ALIGNMENT, CUDA.
  */
 PMLA_API int mla_absorb_query(const uint16_t* q_nope, const uint16_t* q_rope, const uint16_t* w_uk,

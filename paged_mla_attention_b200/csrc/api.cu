@@ -489,7 +489,21 @@ static int proj_call(const uint16_t* a, const uint16_t* rope, const uint16_t* w,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (cr != CUDA_SUCCESS) return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled (weights) failed (%d)", (int)cr);
   }
-  cudaError_t e = pmla::launch_proj(p, absorb, tmap_a, tmap_w, static_cast<cudaStream_t>(stream));
+  // output [tokens][heads][576 or 128] as dims {N, heads, tokens}: a box of 64
+  // columns x 1 head x 32 tokens is one warp's share of a 64-column output group
+  CUtensorMap tmap_out;
+  {
+    const cuuint64_t N = absorb ? 576 : 128;
+    cuuint64_t dim[3] = {N, (cuuint64_t)heads, (cuuint64_t)tokens};
+    cuuint64_t stride[2] = {N * 2, (cuuint64_t)heads * N * 2};
+    cuuint32_t box[3] = {64, 1, 32};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult cr = encode(&tmap_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, out, dim, stride, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return fail(PMLA_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", (int)cr);
+  }
+  cudaError_t e = pmla::launch_proj(p, absorb, tmap_a, tmap_w, tmap_out, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e, "projection kernel launch");
   return PMLA_OK;
 }

@@ -106,7 +106,7 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 cudaError_t launch_clear_counters(int* ctr, int n, cudaStream_t stream);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 cudaError_t launch_proj(const ProjParams& p, bool absorb, const CUtensorMap& tmap_a, const CUtensorMap& tmap_w,
-                        cudaStream_t stream);
+                        const CUtensorMap& tmap_out, cudaStream_t stream);
 size_t decode_smem_bytes();
 
 // Records the message pmla_last_error() returns on this host thread.

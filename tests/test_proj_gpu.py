@@ -38,7 +38,7 @@ def _weights(h, seed):
             _rt(rng.standard_normal((h, 128, 512)) / math.sqrt(512)))
 
 
-@pytest.mark.parametrize("tokens,heads", [(1, 16), (6, 128), (130, 8)])
+@pytest.mark.parametrize("tokens,heads", [(1, 16), (6, 128), (33, 4), (64, 128), (96, 2), (130, 8), (257, 3)])
 def test_projection_kernels_match_fp64(tokens, heads):
     import torch
     import paged_mla_attention_b200 as pm
@@ -61,6 +61,58 @@ def test_projection_kernels_match_fp64(tokens, heads):
     assert np.all(np.abs(q_gpu[..., :512] - q_ref) <= np.abs(q_ref) * 2.0 ** -8 + 1e-4)
     assert np.array_equal(q_gpu[..., 512:], qr)  # the RoPE part passes through
     assert np.all(np.abs(o_gpu - o_ref) <= np.abs(o_ref) * 2.0 ** -8 + 1e-4)
+
+
+def test_rows_past_the_last_token_are_not_written():
+    """The output views end at `tokens`; the rows after them in the same buffer keep
+    their contents (boxes past the end are clipped, not written)."""
+    import torch
+    import paged_mla_attention_b200 as pm
+    T, H = 70, 6
+    rng = np.random.default_rng(3)
+    w_uk, w_uv = _weights(H, 7)
+    q_big = torch.full((T + 60, H, 576), 7.0, dtype=torch.bfloat16, device="cuda")
+    o_big = torch.full((T + 60, H, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    pm.absorb_query(_bf(_rt(rng.standard_normal((T, H, 128)))), _bf(_rt(rng.standard_normal((T, H, 64)))),
+                    _bf(w_uk), out=q_big[:T])
+    pm.project_output(_bf(_rt(rng.standard_normal((T, H, 512)))), _bf(w_uv), out=o_big[:T])
+    torch.cuda.synchronize()
+    assert pm.device_error() == 0
+    assert bool((q_big[T:] == 7.0).all()) and bool((o_big[T:] == 7.0).all())
+    assert not bool((q_big[:T] == 7.0).all())
+
+
+def test_weights_written_by_the_preceding_kernel():
+    """The kernels start before the preceding kernel on the stream has completed
+    (programmatic dependent launch) and prefetch their weights into L2 meanwhile:
+    weights that this preceding kernel writes must still be read as written."""
+    import torch
+    import paged_mla_attention_b200 as pm
+    T, H = 64, 128
+    rng = np.random.default_rng(11)
+    qn = _rt(rng.standard_normal((T, H, 128)))
+    qr = _rt(rng.standard_normal((T, H, 64)))
+    ol = _rt(rng.standard_normal((T, H, 512)))
+    ws = [_weights(H, 20 + i) for i in range(3)]
+    src_uk = [_bf(w[0]) for w in ws]
+    src_uv = [_bf(w[1]) for w in ws]
+    qn_d, qr_d, ol_d = _bf(qn), _bf(qr), _bf(ol)
+    w_uk = torch.empty_like(src_uk[0])
+    w_uv = torch.empty_like(src_uv[0])
+    q = torch.empty((T, H, 576), dtype=torch.bfloat16, device="cuda")
+    o = torch.empty((T, H, 128), dtype=torch.bfloat16, device="cuda")
+    for it in range(6):
+        i = it % 3
+        torch.mul(src_uk[i], 1, out=w_uk)  # a kernel writing the weights, directly before the call
+        pm.absorb_query(qn_d, qr_d, w_uk, out=q)
+        torch.mul(src_uv[i], 1, out=w_uv)
+        pm.project_output(ol_d, w_uv, out=o)
+        q_ref = np.einsum("thk,hkn->thn", qn, ws[i][0])
+        o_ref = np.einsum("thk,hnk->thn", ol, ws[i][1])
+        q_gpu, o_gpu = _np(q), _np(o)
+        assert np.all(np.abs(q_gpu[..., :512] - q_ref) <= np.abs(q_ref) * 2.0 ** -8 + 1e-4), it
+        assert np.all(np.abs(o_gpu - o_ref) <= np.abs(o_ref) * 2.0 ** -8 + 1e-4), it
+    assert pm.device_error() == 0
 
 
 def test_absorbed_pipeline_matches_oracles():
