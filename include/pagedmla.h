@@ -81,6 +81,11 @@ extern "C" {
  *       the shape the metadata is for.
  *   num_parts (out): number of scheduler parts; tile_scheduler_metadata has
  *       num_parts * PMLA_METADATA_INTS int32 entries, num_splits has batch+1.
+ *       One part per decode cluster the device holds at once: with one
+ *       128-row group per KV head a 2-CTA cluster per (part, KV head); with
+ *       more, a 4-CTA cluster per (part, KV head, two row groups), plus the
+ *       parts that 2-CTA clusters (one per row group) run on the SMs the 4-CTA
+ *       clusters leave free (on B200 and num_heads_per_head_k = 256: 33 + 4).
  *   workspace_bytes (out): device workspace mla_decode_with_kvcache needs for
  *       split partial results of this shape (an upper bound over all lengths).
  * Uses the current CUDA device.  Errors: INVALID_ARG, UNSUPPORTED (more than
@@ -103,15 +108,21 @@ PMLA_API int mla_get_metadata_sizes(int batch, int num_heads_per_head_k, int num
  *   tile_scheduler_metadata int32 [num_parts][8], device, out.  Part p covers,
  *       in (sequence, page) order, from (m[0], m[1]) up to but excluding
  *       (m[2], m[3]); m[4] is the ordinal of its first piece among the pieces
- *       of sequence m[0]; m[5..7] are 0.
+ *       of sequence m[0]; m[5] is the part's share weight w_p (128, or 91 for
+ *       a part run by the 2-CTA clusters on the free SMs, which cover a part
+ *       at about 0.71 of the 4-CTA clusters' rate per SM); m[6..7] are 0.
  *   num_splits             int32 [batch+1], device, out: exclusive prefix sum
  *       of pieces per sequence (0 pieces: empty sequence, 1: unsplit).
  *   num_parts              from mla_get_metadata_sizes for the same shape
- *                          (any value in [1, 2048] is accepted).
- * Part boundaries are spaced evenly in cost, assuming every part but the first
- * starts inside a sequence, and snapped so no piece is shorter than two pages;
- * no part costs more than ceil((total + (num_parts-1)*3) / num_parts) + 5,
- * where total sums pages + 3 over the non-empty sequences.
+ *                          (any value in [1, 2048] is accepted; only exactly
+ *                          that value gives parts of weight 91, otherwise all
+ *                          parts weigh 128 and run as 4-CTA clusters).
+ * Part boundaries are spaced in cost in proportion to the weights, assuming
+ * every part but the first starts inside a sequence, and snapped so no piece
+ * is shorter than two pages; no part costs more than
+ * ceil(w_p (total + (num_parts-1)*3) / W) + 5, where total sums pages + 3 over
+ * the non-empty sequences and W sums the weights (with equal weights,
+ * ceil((total + (num_parts-1)*3) / num_parts) + 5).
  * Errors: INVALID_ARG (num_parts outside [1, 2048], null pointers), CUDA.
  */
 PMLA_API int mla_get_metadata(const int32_t* cache_seqlens, int batch, int num_heads_per_head_k,

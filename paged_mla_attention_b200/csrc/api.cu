@@ -59,6 +59,7 @@ struct DeviceInfo {
   bool ready = false;
   int max_clusters = 0;       // 2-CTA decode clusters resident at once
   int max_clusters_pair = 0;  // 4-CTA decode clusters (two row groups each) resident at once
+  int num_sms = 0;
   int* err_ptr = nullptr;
 };
 std::mutex g_mu;
@@ -93,6 +94,7 @@ int device_setup(int* device_out, DeviceInfo** info_out) {
     if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress(device error word)");
     d.max_clusters = n;
     d.max_clusters_pair = n4;
+    d.num_sms = prop.multiProcessorCount;
     d.err_ptr = static_cast<int*>(p);
     d.ready = true;
   }
@@ -121,13 +123,36 @@ int check_shape(int batch, int num_heads_per_head_k, int num_heads_k) {
 
 // Scheduler parts: as many (part, KV head, cluster) work units as decode clusters
 // fit on the device at once.  A KV head with one 128-row group takes one 2-CTA
-// cluster per part; with more, one 4-CTA cluster per two row groups.
-int parts_for(const DeviceInfo& d, int num_heads_per_head_k, int num_heads_k) {
+// cluster per part; with more, one 4-CTA cluster per two row groups, and the
+// SMs those clusters leave free take further parts, each run by one 2-CTA
+// cluster per row group and weighted kPartWeightAux in the schedule.
+struct PartPlan {
+  int main;  // parts of the call's first decode launch
+  int aux;   // parts of the 2-CTA launch on the remaining SMs
+};
+PartPlan part_plan(const DeviceInfo& d, int num_heads_per_head_k, int num_heads_k) {
   const int n_rg = (num_heads_per_head_k + pmla::kRows - 1) / pmla::kRows;
   const bool pair = pmla::decode_uses_pairs(n_rg);
   const long long groups = (long long)(pair ? (n_rg + 1) / 2 : n_rg) * num_heads_k;
   long long parts = (pair ? d.max_clusters_pair : d.max_clusters) / groups;
-  return (int)(parts < 1 ? 1 : parts);
+  if (parts < 1) parts = 1;
+  long long aux = 0;
+  if (pair) {  // SMs left by the 4-CTA clusters, in 2-CTA clusters, one per row group
+    const long long free_sms = (long long)d.num_sms - 4 * parts * groups;
+    aux = free_sms > 0 ? (free_sms / 2) / ((long long)n_rg * num_heads_k) : 0;
+  }
+  return PartPlan{(int)parts, (int)aux};
+}
+int parts_for(const DeviceInfo& d, int num_heads_per_head_k, int num_heads_k) {
+  const PartPlan pl = part_plan(d, num_heads_per_head_k, num_heads_k);
+  return pl.main + pl.aux;
+}
+// Parts of the first decode launch for a call with num_parts parts: all of them
+// unless num_parts is exactly what part_plan gives (the schedule then weighs
+// the rest kPartWeightAux and they run as the 2-CTA launch).
+int main_parts(const DeviceInfo& d, int num_heads_per_head_k, int num_heads_k, int num_parts) {
+  const PartPlan pl = part_plan(d, num_heads_per_head_k, num_heads_k);
+  return (pl.aux > 0 && num_parts == pl.main + pl.aux) ? pl.main : num_parts;
 }
 
 size_t workspace_for(int batch, int R, int h_kv, int num_parts, size_t* lse_offset) {
@@ -190,7 +215,12 @@ int mla_get_metadata(const int32_t* cache_seqlens, int batch, int num_heads_per_
     return fail(PMLA_ERR_INVALID_ARG, "null pointer argument");
   if (num_parts < 1 || num_parts > pmla::kMaxParts)
     return fail(PMLA_ERR_INVALID_ARG, "num_parts %d outside [1, %d]", num_parts, pmla::kMaxParts);
-  cudaError_t e = pmla::launch_metadata(cache_seqlens, batch, num_parts, tile_scheduler_metadata,
+  int dev;
+  DeviceInfo* d;
+  rc = device_setup(&dev, &d);
+  if (rc) return rc;
+  const int num_main = main_parts(*d, num_heads_per_head_k, num_heads_k, num_parts);
+  cudaError_t e = pmla::launch_metadata(cache_seqlens, batch, num_parts, num_main, tile_scheduler_metadata,
                                         num_splits, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail_cuda(e, "metadata kernel launch");
   return PMLA_OK;
@@ -340,6 +370,8 @@ int decode_impl(const uint16_t* q, const uint16_t* kvcache, const int32_t* block
     p.R = (int)R;
     p.n_rg = (int)((R + pmla::kRows - 1) / pmla::kRows);
     p.num_parts = num_parts;
+    p.part0 = 0;
+    p.follows_decode = 0;
     p.max_pages = max_pages_per_seq;
     p.num_pages = num_pages;
     p.causal = causal ? 1 : 0;
@@ -353,8 +385,18 @@ int decode_impl(const uint16_t* q, const uint16_t* kvcache, const int32_t* block
     // the merge kernel counts completion signals from zero
     e = pmla::launch_clear_counters(p.seq_done, (int)wl.done_count, st);
     if (e != cudaSuccess) return fail_cuda(e, "clearing the completion counters");
-    e = pmla::launch_decode(p, tmap, tmap_q, tmap_v, tmap_kv2, pair, st);
+    const int num_main = main_parts(*info, (int)R, h_kv, num_parts);
+    e = pmla::launch_decode(p, tmap, tmap_q, tmap_v, tmap_kv2, pair, num_main, st);
     if (e != cudaSuccess) return fail_cuda(e, "decode kernel launch");
+    if (num_main < num_parts) {
+      // the remaining parts on the SMs the 4-CTA clusters leave free: 2-CTA
+      // clusters, one per row group, launched as a programmatic dependent of
+      // the first decode kernel (they start once all of its CTAs are resident)
+      p.part0 = num_main;
+      p.follows_decode = 1;
+      e = pmla::launch_decode(p, tmap, tmap_q, tmap_v, tmap_kv2, false, num_parts - num_main, st);
+      if (e != cudaSuccess) return fail_cuda(e, "decode kernel launch (remaining SMs)");
+    }
   }
   if (!(stages & kStageMerge)) return PMLA_OK;
 

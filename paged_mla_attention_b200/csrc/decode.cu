@@ -277,6 +277,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
   const int warp = tid >> 5, lane = tid & 31;
   if (sbase & 1023u) {  // layout assumption broken: report and leave (uniform branch)
     if (tid == 0) atomicCAS(P.err, 0, kErrBadSmemAlign);
+    if (P.follows_decode && blockIdx.x == 0 && tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
     return;
   }
   constexpr int kClusterCtas = kPair ? 4 : 2;
@@ -291,7 +292,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
   const int cluster_id = blockIdx.x / kClusterCtas;
   const int units = kPair ? (P.n_rg + 1) / 2 : P.n_rg;  // clusters per KV head and part
   const int groups = P.h_kv * units;
-  const int part = cluster_id / groups;
+  const int part = P.part0 + cluster_id / groups;
   const int g = (cluster_id % groups) / units;
   const int rg = kPair ? 2 * ((cluster_id % groups) % units) + (int)half : (cluster_id % groups) % units;
 
@@ -363,11 +364,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
   const uint32_t tmem = ctrl->tmem_base;
   // launched as a programmatic dependent of the counter clear: the setup above
   // overlaps the kernels before it; the schedule and the cleared counters are
-  // read only after this wait (the clear's grid completes after the schedule's)
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  // every CTA of this grid is resident now: the merge kernel, launched as a
-  // programmatic dependent, may start on SMs as they free up (it waits for the
-  // completion signals of the pieces it merges)
+  // read only after this wait (the clear's grid completes after the schedule's).
+  // A decode launch that follows the call's first decode kernel (the 2-CTA
+  // clusters on the SMs the 4-CTA clusters leave free) skips it: it is launched
+  // only once every CTA of that kernel has passed this wait and triggered, so
+  // the schedule and the clear have completed, and waiting here would wait for
+  // that whole kernel.
+  if (!P.follows_decode) asm volatile("griddepcontrol.wait;" ::: "memory");
+  // every CTA of this grid is resident now: the next kernel (the merge, or the
+  // second decode launch), launched as a programmatic dependent, may start on
+  // SMs as they free up (the merge waits for the completion signals of the
+  // pieces it merges)
   if (tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const PartIter it(P, part);
   // the CTA on the other side of the P hand-off (S-CTA <-> O-CTA of a row group)
@@ -1291,6 +1298,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant
     else
       tmem_dealloc(tmem, 512);
   }
+  // a second decode launch completes only after the first (one CTA waits for
+  // it), so that the merge grid's completion, which waits for this grid's, also
+  // implies the first's: work queued after the call sees every output row
+  if (P.follows_decode && blockIdx.x == 0 && tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace
@@ -1332,11 +1343,11 @@ int decode_max_active_clusters(int device, bool pair, int* out) {
 }
 
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, const CUtensorMap& tmap_q,
-                          const CUtensorMap& tmap_v, const CUtensorMap& tmap_kv2, bool pair,
+                          const CUtensorMap& tmap_v, const CUtensorMap& tmap_kv2, bool pair, int parts,
                           cudaStream_t stream) {
   const int ctas = pair ? 4 : 2;
   const int units = pair ? (p.n_rg + 1) / 2 : p.n_rg;
-  const int clusters = p.num_parts * p.h_kv * units;
+  const int clusters = parts * p.h_kv * units;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas * clusters, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

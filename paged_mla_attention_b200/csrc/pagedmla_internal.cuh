@@ -21,6 +21,16 @@ constexpr int kMaxParts = 2048; // scheduler parts one metadata kernel handles
 // write and its re-read by the merge kernel.
 constexpr int kPieceCostPages = 3;
 
+// Share weights of scheduler parts (tile_scheduler_metadata column 5).  With
+// two or more row groups per KV head the parts run on 4-CTA clusters of the
+// pair variant, which leave some SMs free (148 - 4 x 33 = 16 on B200); those
+// take 2-CTA clusters of the one-row-group variant, one per row group of a
+// part, which cover a part at about 0.71 of the pair variant's rate per SM
+// (measured: 0.39 of the bf16 peak on 148 SMs against 0.49 on 132), so their
+// parts get that share of the work.
+constexpr int kPartWeightFull = 128;
+constexpr int kPartWeightAux = 91;  // best of 80 / 91 / 102 / 112 on the causal2 workload
+
 // Device error codes written by bounded waits that time out (first one wins).
 enum DeviceError : int {
   kErrNone = 0,
@@ -48,6 +58,8 @@ struct DecodeParams {
   int R;                        // s_q * hpk rows per KV head
   int n_rg;                     // ceil(R / 128) row groups
   int num_parts, max_pages, num_pages, causal;
+  int part0;                    // first scheduler part of this launch
+  int follows_decode;           // 1: launched after the call's other decode kernel (see the kernel)
   float scale_log2;             // softmax_scale * log2(e)
 };
 
@@ -91,7 +103,8 @@ struct WorkspaceLayout {
 WorkspaceLayout workspace_layout(int batch, int R, int h_kv, int num_parts);
 
 // Host launchers (each returns the CUDA error of its launch).
-cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* meta,
+// Parts [0, num_main) weigh kPartWeightFull, the others kPartWeightAux.
+cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int num_main, int32_t* meta,
                             int32_t* num_splits, cudaStream_t stream);
 cudaError_t decode_prepare(int device);  // one-time per-device kernel attributes
 // Clusters of the decode kernel resident at once: 2-CTA clusters (pair = false,
@@ -99,8 +112,9 @@ cudaError_t decode_prepare(int device);  // one-time per-device kernel attribute
 int decode_max_active_clusters(int device, bool pair, int* out);
 // The 4-CTA variant is used when a KV head has two or more row groups.
 inline bool decode_uses_pairs(int n_rg) { return n_rg >= 2; }
+// Launches the clusters of parts [p.part0, p.part0 + parts).
 cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_kv, const CUtensorMap& tmap_q,
-                          const CUtensorMap& tmap_v, const CUtensorMap& tmap_kv2, bool pair,
+                          const CUtensorMap& tmap_v, const CUtensorMap& tmap_kv2, bool pair, int parts,
                           cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream);
 cudaError_t launch_clear_counters(int* ctr, int n, cudaStream_t stream);

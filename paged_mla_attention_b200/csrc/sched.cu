@@ -11,18 +11,21 @@
 //                        position (b, page) sits at X = S_b + F + page, the
 //                        start of sequence b at X = S_b
 //   total              = S_batch
-//   boundary of part p = X_p = floor(p (total + (P-1) F) / P) - (p-1) F
+//   weights            = w_p = kPartWeightFull for parts p < num_main,
+//                        kPartWeightAux after (parts run by slower clusters);
+//                        C_p = w_0 + ... + w_{p-1}, W = C_P
+//   boundary of part p = X_p = floor(C_p (total + (P-1) F) / W) - (p-1) F
 //
 // Every part is assumed to start inside a sequence and so pay one F of its
-// own; the spacing of the X_p gives each part the same share of the total plus
-// those P-1 overheads.  X_p is mapped back to (b, page) and snapped so that no
+// own; the spacing of the X_p gives each part its weight's share of the total
+// plus those P-1 overheads (with equal weights, p (total + (P-1) F) / P).  X_p is mapped back to (b, page) and snapped so that no
 // piece is shorter than two pages: a start at page 1 moves to the sequence
 // start, a start that would leave a one-page tail moves to the next sequence.
 // Snapping is monotone, so parts stay ordered (some may be empty).  When the
 // whole batch costs less than P (F + 1) the overhead assumption is dropped and
-// X_p = floor(p total / P).
+// X_p = floor(C_p total / W).
 //
-// A part's cost is at most ceil((total + (P-1) F) / P) + F + 2 in either
+// A part's cost is at most ceil(w_p (total + (P-1) F) / W) + F + 2 in either
 // regime; each thread finds its boundary by binary search, so the kernel
 // takes a few microseconds for any batch.
 #include "pagedmla_internal.cuh"
@@ -70,7 +73,7 @@ __device__ long long block_exclusive_scan(long long v, long long* warp_tot, long
 }  // namespace
 
 __global__ void __launch_bounds__(kSchedThreads) metadata_kernel(const int32_t* __restrict__ seqlens,
-                                                                 int batch, int num_parts,
+                                                                 int batch, int num_parts, int num_main,
                                                                  int32_t* __restrict__ meta,
                                                                  int32_t* __restrict__ num_splits) {
   __shared__ long long chunk_base[kSchedThreads];  // cost coordinate of each chunk's first sequence
@@ -106,16 +109,19 @@ __global__ void __launch_bounds__(kSchedThreads) metadata_kernel(const int32_t* 
   chunk_ne[t] = (int)block_exclusive_scan(cne, warp_tot, &sh_scratch);
   const long long total = sh_total;  // the scans end with a barrier
 
-  // 2. part boundaries
+  // 2. part boundaries (C_p <= 2^11 x 2^7 and A < 2^42: the products fit 64 bits)
   const long long A = total + (long long)(P - 1) * F;
   const bool overhead_model = A >= (long long)P * (F + 1);
+  const int M = min(max(num_main, 0), P);
+  const int W = M * kPartWeightFull + (P - M) * kPartWeightAux;
+  const long long span = overhead_model ? A : total;
   for (int p = t; p <= P; p += kSchedThreads) {
     int sb = batch, spg = 0;
     if (p == 0) {
       sb = 0;
     } else if (p < P) {
-      const long long X = overhead_model ? (long long)p * A / P - (long long)(p - 1) * F
-                                         : (long long)p * total / P;
+      const int cw = p <= M ? p * kPartWeightFull : M * kPartWeightFull + (p - M) * kPartWeightAux;
+      const long long X = (long long)cw * span / W - (overhead_model ? (long long)(p - 1) * F : 0);
       if (X < total) {
         // last chunk whose base is <= X (its cost is > 0 because X < total)
         int lo = 0, hi = kSchedThreads - 1;
@@ -191,7 +197,7 @@ __global__ void __launch_bounds__(kSchedThreads) metadata_kernel(const int32_t* 
     m[2] = start_b[p + 1];
     m[3] = start_pg[p + 1];
     m[4] = pg0 > 0 ? cut_rank[p] - cuts_before(b0, false) : 0;
-    m[5] = 0;
+    m[5] = p < M ? kPartWeightFull : kPartWeightAux;
     m[6] = 0;
     m[7] = 0;
   }
@@ -208,9 +214,9 @@ __global__ void __launch_bounds__(kSchedThreads) metadata_kernel(const int32_t* 
   }
 }
 
-cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* meta,
+cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int num_main, int32_t* meta,
                             int32_t* num_splits, cudaStream_t stream) {
-  metadata_kernel<<<1, kSchedThreads, 0, stream>>>(seqlens, batch, num_parts, meta, num_splits);
+  metadata_kernel<<<1, kSchedThreads, 0, stream>>>(seqlens, batch, num_parts, num_main, meta, num_splits);
   return cudaGetLastError();
 }
 
