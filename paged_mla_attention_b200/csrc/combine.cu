@@ -11,12 +11,12 @@
 // unsplit sequences (n = 1) were written by the decode kernel directly.
 //
 // Layout: the partials are chunk-major, [slot][h_kv][64 chunks of 8 columns]
-// [R rows][8].  A block takes 32 consecutive rows and one eighth (64) of the
-// columns of one (sequence, KV head); warp w handles chunk w of that slice,
-// lane = row, so every load is 1 KB contiguous, and 8 pieces' loads are in
-// flight at once.  The merged rows go through shared memory and leave as
-// contiguous 16-byte stores.  Grid: (row blocks of 32 x 8 column slices, h_kv,
-// batch).
+// [R rows][8].  A block takes 32 consecutive rows and one column slice (all
+// 512 columns, a quarter or an eighth) of one (sequence, KV head); warps take
+// the chunks of that slice, lane = row, so every load is 1 KB contiguous, with
+// the loads of several pieces in flight at once.  The merged rows go through
+// shared memory and leave as contiguous 16-byte stores.  Grid: (row blocks of
+// 32 x column slices, h_kv, batch).
 //
 // Overlap with the decode kernel: this kernel is launched as a programmatic
 // dependent of the decode kernel, which lets it start once every decode CTA is
@@ -260,9 +260,15 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
   if (p.batch == 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
   // a long sequence cut into many pieces shows as many scheduler parts per
-  // sequence: spread each row block over 8 column slices then
+  // sequence: spread each row block over 8 column slices then.  Otherwise a
+  // sequence has a few pieces (mostly two, the halves of a cut): with one row
+  // group per KV head, 4 column slices with both pieces' loads in flight at once
+  // (the tail after the decode kernel: uniform 11.0 -> 6.5 us, varlen 17.3 ->
+  // 7.8 us); with more row groups one block per row block (4 slices measured no
+  // better on causal2).
   const bool many = p.num_parts >= 2 * p.batch;
-  const int slices = many ? 8 : 1;
+  const bool sliced = !many && p.R <= kRows;
+  const int slices = many ? 8 : sliced ? 4 : 1;
   cfg.gridDim = dim3(((p.R + kMergeRows - 1) / kMergeRows) * slices, p.h_kv, p.batch);
   cfg.blockDim = dim3(many ? 2 * kMergeThreads : kMergeThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
@@ -272,8 +278,8 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return many ? cudaLaunchKernelEx(&cfg, combine_kernel<8, 8, 2>, p)
-              : cudaLaunchKernelEx(&cfg, combine_kernel<1, 1>, p);
+  if (many) return cudaLaunchKernelEx(&cfg, combine_kernel<8, 8, 2>, p);
+  return sliced ? cudaLaunchKernelEx(&cfg, combine_kernel<4, 2>, p) : cudaLaunchKernelEx(&cfg, combine_kernel<1, 1>, p);
 }
 
 }  // namespace pmla
