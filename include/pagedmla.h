@@ -108,14 +108,14 @@ PMLA_API int mla_get_metadata_sizes(int batch, int num_heads_per_head_k, int num
  *   tile_scheduler_metadata int32 [num_parts][8], device, out.  Part p covers,
  *       in (sequence, page) order, from (m[0], m[1]) up to but excluding
  *       (m[2], m[3]); m[4] is the ordinal of its first piece among the pieces
- *       of sequence m[0]; m[5] is the part's share weight w_p (128, or 91 for
- *       a part run by the 2-CTA clusters on the free SMs, which cover a part
- *       at about 0.71 of the 4-CTA clusters' rate per SM); m[6..7] are 0.
+ *       of sequence m[0]; m[5] is the part's share weight w_p (128, or 107
+ *       for a part run by the 2-CTA clusters on the free SMs, which cover a
+ *       part at about 0.84 of the 4-CTA clusters' rate per SM); m[6..7] are 0.
  *   num_splits             int32 [batch+1], device, out: exclusive prefix sum
  *       of pieces per sequence (0 pieces: empty sequence, 1: unsplit).
  *   num_parts              from mla_get_metadata_sizes for the same shape
  *                          (any value in [1, 2048] is accepted; only exactly
- *                          that value gives parts of weight 91, otherwise all
+ *                          that value gives parts of weight 107, otherwise all
  *                          parts weigh 128 and run as 4-CTA clusters).
  * Part boundaries are spaced in cost in proportion to the weights, assuming
  * every part but the first starts inside a sequence, and snapped so no piece

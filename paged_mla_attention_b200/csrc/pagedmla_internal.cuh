@@ -25,11 +25,12 @@ constexpr int kPieceCostPages = 3;
 // two or more row groups per KV head the parts run on 4-CTA clusters of the
 // pair variant, which leave some SMs free (148 - 4 x 33 = 16 on B200); those
 // take 2-CTA clusters of the one-row-group variant, one per row group of a
-// part, which cover a part at about 0.71 of the pair variant's rate per SM
-// (measured: 0.39 of the bf16 peak on 148 SMs against 0.49 on 132), so their
-// parts get that share of the work.
+// part.  Running beside the 4-CTA clusters they cover a part at about 0.84 of
+// their rate per SM, so their parts get that share of the work (on causal2,
+// per-cluster end times: weight 91 left them idle for the last ~50 us of
+// ~365 us, 107 ends both kinds of cluster within ~2 us of each other).
 constexpr int kPartWeightFull = 128;
-constexpr int kPartWeightAux = 91;  // best of 80 / 91 / 102 / 112 on the causal2 workload
+constexpr int kPartWeightAux = 107;
 
 // Device error codes written by bounded waits that time out (first one wins).
 enum DeviceError : int {
