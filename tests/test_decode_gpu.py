@@ -81,6 +81,19 @@ def test_split_sequences_merge():
     assert np.diff(splits).max() >= 2, "expected at least one split sequence"
 
 
+@pytest.mark.parametrize("lens,s_q,h_q,h_kv,causal", [
+    ([5000, 64], 2, 128, 1, True),        # two row groups per KV head (4-CTA clusters)
+    ([12000, 200, 5], 1, 64, 2, False),   # two KV heads
+    ([2200, 2200, 1], 1, 128, 1, False),  # two long sequences sharing the parts
+])
+def test_merge_of_many_pieces(lens, s_q, h_q, h_kv, causal):
+    # few sequences, one or two of them long: more than 16 pieces each, merged by the
+    # many-piece variant (8 column slices, two groups of warps taking pieces in turns)
+    stats, meta, splits = _check(_small(lens, s_q=s_q, h_q=h_q, h_kv=h_kv, causal=causal, seed=sum(lens) % 97),
+                                 f"many pieces {lens}")
+    assert np.diff(splits).max() > 16, f"expected a sequence in more than 16 pieces, got {np.diff(splits)}"
+
+
 def test_grouped_kv_heads():
     _check(_small([70, 300, 5], s_q=1, h_q=32, h_kv=2, seed=23), "h_kv=2")
     _check(_small([129, 40], s_q=2, h_q=64, h_kv=4, causal=True, seed=24), "h_kv=4 causal")
