@@ -17,13 +17,14 @@
 //             W 16 KB each) through a ring of slots.
 // At decode sizes (a step's tokens are at most a few hundred) the kernels are
 // bound by reading the weights (128 KB per head) and moving the activations.
-// With several token tiles, two CTAs fit an SM (96 KB of shared memory and at
-// most 256 TMEM columns each), so one CTA's epilogue overlaps the other's
-// loads; with one tile (at most 128 tokens) the unabsorb grid is one CTA per
-// head, fewer than the SMs, and its ring has six slots (192 KB) so that six of
-// the eight chunks are in flight at once.  Results leave through shared memory by TMA stores (one
-// 32-token x 64-column box per warp), which write whole 128-byte rows; tokens
-// past the end read as zeros and are not stored.
+// Absorb CTAs, and unabsorb CTAs when there are several token tiles, take 96 KB
+// of shared memory and at most 256 TMEM columns, so two fit an SM and one's
+// epilogue overlaps the other's loads; with one tile (at most 128 tokens) the
+// unabsorb grid is one CTA per head, fewer than the SMs, and its ring has six
+// slots (192 KB) so that six of the eight chunks are in flight at once.
+// Results leave through shared memory by TMA stores (one 32-token x 64-column
+// box per warp), which write whole 128-byte rows; tokens past the end read as
+// zeros and are not stored.
 //
 // The kernels are launched as programmatic dependents of the preceding kernel
 // on the stream: a CTA sets up, lets its own dependents launch, and prefetches
