@@ -1,8 +1,9 @@
 """Planted mistakes in copies of the oracle must each fail at least one pin.
 
 Each mutant is the oracle's C source with one plausible error written in
-(a dropped scale, an off-by-one mask, the wrong value columns, a wrong page or
-head index, a dropped max in lse, a sign slip in the merge).  The copy is
+(a dropped scale, an off-by-one or reversed mask, the wrong value columns, a
+wrong page or head index, a dropped max or the wrong base in lse, unnormalised
+weights, a sign slip or a dropped part in the merge).  The copy is
 compiled on the CPU into a temporary directory; the real oracle is untouched.
 """
 import os
@@ -31,6 +32,20 @@ MUTANTS = {
     "unabsorbed_wv_transposed": ("t += wv[(size_t)r * dc + k] * c[k];", "t += wv[(size_t)k * dvo + r] * c[k];"),
     "unabsorbed_rope_dropped": ("for (int r = 0; r < dr; ++r) acc += qr[r] * c[dc + r];",
                                 "for (int r = 0; r < dr; ++r) acc += 0.0 * qr[r] * c[dc + r];"),
+    "causal_query_reversed": ("int last = causal ? L - s_q + i : L - 1;",
+                              "int last = causal ? L - 1 - i : L - 1;"),
+    "non_causal_drops_last": ("int last = causal ? L - s_q + i : L - 1;",
+                              "int last = causal ? L - s_q + i : L - 2;"),
+    "lse_base_2": ("*lse_out = m + log(z);", "*lse_out = m + log2(z);"),
+    "weights_unnormalised": ("const double w = exp(s[j - first] - m) / z;",
+                             "const double w = exp(s[j - first] - m);"),
+    "empty_row_lse_zero": ("*lse_out = -INFINITY;\n      continue;", "*lse_out = 0.0;\n      continue;"),
+    "value_head_zero": ("const uint16_t* vrow = kv_row(kv, block_table, max_pages, b, j, g, h_kv, d, page_size);",
+                        "const uint16_t* vrow = kv_row(kv, block_table, max_pages, b, j, 0, h_kv, d, page_size);"),
+    "window_end_off_by_one": ("if (key_hi && key_hi[b] - 1 < last) last = key_hi[b] - 1;",
+                              "if (key_hi && key_hi[b] - 1 < last) last = key_hi[b];"),
+    "merge_skips_first_part": ("for (int k = 0; k < n; ++k) {\n    const double w = exp(part_lse[k] - total);",
+                               "for (int k = 1; k < n; ++k) {\n    const double w = exp(part_lse[k] - total);"),
     "append_head": ("uint16_t* dst =\n            kvcache + (((size_t)page * page_size + (size_t)(pos % page_size)) * h_kv + g)",
                     "uint16_t* dst =\n            kvcache + (((size_t)page * page_size + (size_t)(pos % page_size)) * h_kv + 0)"),
 }
